@@ -1,0 +1,225 @@
+/*
+ * sa.h - C ABI of a B200 (sm_100a) library for block-sparse attention driven
+ * by a per-input mask: per-input block selection, per-(layer, head) head
+ * skipping, and flash-style attention over only the selected tiles.
+ *
+ * Sources the operations follow (web pages describing the method):
+ *   [SDN] SD.Next ("automatic") commit log for modules/attention/sparse:
+ *         the "selector", "layout", "radial control", "host sync" and
+ *         "flex consumer" paragraphs.
+ *   [HS]  haagenti_sparse crate (docs.rs overview and lib.rs): AttentionMask,
+ *         SparseKernel, SparseError, MIN_ACTIVE_HEADS = 4,
+ *         DEFAULT_SPARSITY = 0.5.
+ *   [GLO] inferensys glossary "Sparse Attention": sliding window, dilated,
+ *         global and block-sparse patterns; CSR rows.
+ *
+ * Conventions shared by every call:
+ *   - Tensors Q, K, V, O are bf16, row-major [B][H][N][d] on the device,
+ *     contiguous, 16-byte aligned.  d is 64 or 128; N is a multiple of the
+ *     block size (64).  nB = N / 64 blocks per head.
+ *   - The caller owns every device buffer.  The library owns only layouts
+ *     (sa_layout), which hold small device arrays allocated once per layout.
+ *   - Hot calls (sa_select_blocks, sa_pattern_mask, sa_block_sparse_attention,
+ *     sa_dense_attention) never allocate, never synchronise the host and
+ *     never read device memory back; they enqueue kernels on `stream`.
+ *   - Argument and shape errors are returned before anything is launched.
+ *     Faults found on the device (an out-of-range block index, a bounded
+ *     wait that ran out) set a sticky error word in the workspace header and
+ *     the kernel skips the bad access; sa_check() reads and clears it.
+ *   - Block lists are CSR-like rows of fixed capacity [GLO CSR]:
+ *     idx[b][h][i][0 .. counts[b][h][i]) holds the kept key blocks of query
+ *     block i in ascending order; slots at or beyond the count are left
+ *     untouched and are unspecified.
+ *   - head_mask is a HOST array of H bytes (nonzero = compute the head)
+ *     [HS AttentionMask], or NULL for all heads.  H <= 64.  Fewer than
+ *     min_active active heads is SA_ERR_HEAD_MASK [HS MIN_ACTIVE_HEADS];
+ *     a skipped head gets counts 0 and O = 0.
+ */
+#ifndef SA_H_
+#define SA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers. */
+typedef struct CUstream_st* sa_stream_t;
+
+/* Error codes [HS SparseError]. */
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,  /* null pointer, bad enum, density outside (0, 1]   */
+  SA_ERR_SHAPE = 2,        /* d not 64/128, N not a multiple of 64, B/H <= 0    */
+  SA_ERR_LAYOUT = 3,       /* segments do not tile [0, N) in order               */
+  SA_ERR_HEAD_MASK = 4,    /* fewer than min_active heads active                 */
+  SA_ERR_WORKSPACE = 5,    /* workspace missing or smaller than sa_workspace_size */
+  SA_ERR_BAD_INDEX = 6,    /* device: a block index outside [0, nB) or count > cap */
+  SA_ERR_TIMEOUT = 7,      /* device: a bounded wait inside a kernel ran out     */
+  SA_ERR_UNSUPPORTED = 8,  /* not a B200-class (sm_100) device                   */
+  SA_ERR_CUDA = 9          /* a CUDA runtime call failed                         */
+} sa_status;
+
+/* Token segment kinds [SDN "layout"]: image/video tokens are sparsifiable;
+ * text, conditioning, audio and unknown tokens pin their rows and columns;
+ * padding is dropped. */
+typedef enum {
+  SA_SEG_TEXT = 0,   /* live prompt conditioning: pinned   */
+  SA_SEG_PAD = 1,    /* padding: dropped                   */
+  SA_SEG_IMAGE = 2,  /* image / video tokens: sparsifiable */
+  SA_SEG_OTHER = 3   /* audio / unrecognised: pinned       */
+} sa_seg_kind;
+
+typedef struct {
+  int32_t kind;   /* sa_seg_kind                 */
+  int32_t start;  /* first token of the run      */
+  int32_t len;    /* tokens in the run (> 0)     */
+} sa_segment;
+
+/* Block classes a layout assigns (exposed for tests and tools). */
+typedef enum { SA_BLOCK_PIN = 0, SA_BLOCK_SPARSE = 1, SA_BLOCK_DROP = 2 } sa_block_class;
+
+typedef struct sa_layout sa_layout;  /* opaque, library-owned, refcounted, cached */
+
+/* Control patterns [SDN "radial control"; GLO sliding window, dilated, global]. */
+typedef enum { SA_PAT_RADIAL = 0, SA_PAT_WINDOW_GLOBAL = 1, SA_PAT_DILATED = 2 } sa_pattern_kind;
+
+typedef struct {
+  int32_t kind;             /* sa_pattern_kind                                        */
+  int32_t window_tokens;    /* W: keys with |q - key| <= W (window, dilated)          */
+  int32_t n_global_blocks;  /* G: the first G sparsifiable blocks are global rows and
+                               columns (window and dilated patterns)                  */
+  int32_t dilation;         /* r: dilated keys satisfy (q - key) % r == 0 (r >= 1)    */
+} sa_pattern;
+
+/* Optional per-call statistics [HS KernelStats]: filled only by sa_density. */
+typedef struct {
+  double density_over_active;  /* sum(counts) / (B * H_active * nB^2) */
+  double density_over_all;     /* sum(counts) / (B * H * nB^2)        */
+  int64_t tiles;               /* sum(counts) over active heads       */
+  int32_t heads_active;        /* active heads in the mask            */
+} sa_stats;
+
+/*
+ * sa_build_layout [SDN "layout" paragraph; the geometry "built once and
+ * cached per layout" of the "host sync" paragraph].
+ *   segs/nseg: runs that tile [0, N) in order (nseg == 0: the whole sequence
+ *   is sparsifiable, as when a pipeline publishes no layout).  N % block == 0,
+ *   block must be 64.  A block is PIN if it holds text/other tokens or mixes
+ *   kinds (a tile straddling a boundary pins), DROP if it is all padding,
+ *   SPARSE if it is all image.  *out receives a refcounted handle; an
+ *   identical (N, block, segments) request returns the cached layout with its
+ *   count raised.  May allocate and synchronise (once per layout, outside the
+ *   hot loop).  Release with sa_layout_release.
+ */
+sa_status sa_build_layout(const sa_segment* segs, int nseg, int N, int block, sa_layout** out);
+
+/* nB blocks, n_pin / n_drop / n_cand (= C, sparsifiable) blocks, and cap =
+ * nB - n_drop, the capacity an idx row needs.  Any output pointer may be NULL. */
+sa_status sa_layout_info(const sa_layout* L, int* nB, int* n_pin, int* n_drop, int* n_cand, int* cap);
+
+/* Host copy of the per-block classes (sa_block_class), nB bytes. */
+sa_status sa_layout_classes(const sa_layout* L, uint8_t* cls_out, int nB);
+
+/* Drops one reference; the layout is freed when the count reaches zero. */
+sa_status sa_layout_release(sa_layout* L);
+
+/* Budget in kept candidates per sparse row [SDN "selector": a fraction of the
+ * sparsifiable candidates]: clamp(floor(density * C + 1e-4), 1, C). */
+int sa_budget(float density, int n_cand);
+
+/*
+ * sa_select_blocks [SDN "selector" + "host sync" paragraphs].
+ * Per (batch, active head, 64-row query block i):
+ *   qbar_i = mean of the 64 Q rows, kbar_j likewise (fp32 accumulation);
+ *   s_ij = qbar_i . kbar_j in fp32, with no scale and no softmax;
+ *   a SPARSE row keeps its diagonal block, then the k-1 highest-scoring
+ *   other SPARSE blocks (ties: lower block index; -0 ranks as +0), plus every
+ *   PIN block; k = sa_budget(density, C).  A PIN row keeps every non-DROP
+ *   block; a DROP row keeps nothing.  Lists are emitted in ascending order.
+ * The rank is found on the device (no host-sized top-k, no readback).  When
+ * k == C the budget covers every candidate and the call writes the dense
+ * lists without pooling or scoring (unless scores_out is requested).
+ *   Q, K:       device bf16 [B][H][N][d].
+ *   idx:        device int32 [B][H][nB][cap]; counts: device int32 [B][H][nB].
+ *   scores_out: device fp32 [B][H][nB][nB] or NULL; when given, every active
+ *               head's scores are written (rows of inactive heads untouched).
+ *   ws:         device workspace of at least sa_workspace_size bytes,
+ *               header zeroed once with sa_workspace_init.
+ */
+sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void* K, int B, int H, int d,
+                           float density, const uint8_t* head_mask, int min_active,
+                           int32_t* idx, int32_t* counts, float* scores_out,
+                           void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/*
+ * sa_pattern_mask [SDN "radial control"; GLO sliding window / dilated /
+ * global].  Writes the same (idx, counts) a selection would, from a fixed
+ * pattern honouring the same pins and drops:
+ *   RADIAL: the selector's k = sa_budget(density, C) SPARSE blocks nearest to
+ *     the diagonal (distance |i - j|, ties to the lower j).
+ *   WINDOW_GLOBAL: SPARSE blocks j with some token pair |q - key| <= W
+ *     between blocks i and j, plus the first G SPARSE blocks as global
+ *     columns; those G blocks' rows are dense over non-DROP blocks.
+ *   DILATED: SPARSE blocks holding some key with |q - key| <= W and
+ *     (q - key) % r == 0 for some query of block i, plus G globals as above.
+ * density is used by RADIAL only.  No workspace needed.
+ */
+sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H, float density,
+                          const uint8_t* head_mask, int min_active,
+                          int32_t* idx, int32_t* counts, sa_stream_t stream);
+
+/*
+ * sa_block_sparse_attention [GLO block-sparse; SDN "flex consumer": every
+ * selected tile is computed in full].  For each active head and query row q
+ * of block i:  O_q = softmax(Q_q . K_S^T * scale) . V_S, with S the tokens of
+ * the blocks idx[b][h][i][0 .. counts) (online softmax, fp32 accumulation,
+ * bf16 MMA on tcgen05).  Rows with count 0 and skipped heads get O = 0.
+ *   idx/counts/cap: as written by sa_select_blocks or sa_pattern_mask; any
+ *     index outside [0, nB) or count > cap sets SA_ERR_BAD_INDEX on the
+ *     device and the entry is skipped.
+ *   softmax_scale: 0 means 1/sqrt(d).
+ *   O: device bf16 [B][H][N][d], fully written.
+ */
+sa_status sa_block_sparse_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                    const int32_t* idx, const int32_t* counts, int cap,
+                                    const uint8_t* head_mask, int min_active, float softmax_scale,
+                                    void* O, void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* sa_dense_attention: the same kernel over every tile of every head (the
+ * dense baseline the speedup is measured against). */
+sa_status sa_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                             float softmax_scale, void* O, void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/*
+ * sa_density [SDN "host sync": density is read back only when something
+ * asks].  The only call that reads device memory back: it synchronises
+ * `stream`.  Any of the outputs may be NULL.
+ */
+sa_status sa_density(const int32_t* counts, int B, int H, int nB, const uint8_t* head_mask,
+                     double* over_active, double* over_all, sa_stats* stats,
+                     void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* Workspace bytes needed by every call for these sizes (selection and
+ * attention regions are disjoint, so one workspace serves both). */
+sa_status sa_workspace_size(int B, int H, int N, int d, size_t* bytes);
+
+/* Zeroes the workspace header (the sticky error word); enqueued on stream. */
+sa_status sa_workspace_init(void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the workspace error word, and
+ * returns SA_OK or the first device-side error recorded. */
+sa_status sa_check(void* ws, sa_stream_t stream);
+
+const char* sa_status_string(sa_status s);
+
+/* Library version string. */
+const char* sa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_H_ */
