@@ -41,6 +41,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define SA_API __attribute__((visibility("default")))
+#else
+#define SA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -114,21 +120,21 @@ typedef struct {
  *   count raised.  May allocate and synchronise (once per layout, outside the
  *   hot loop).  Release with sa_layout_release.
  */
-sa_status sa_build_layout(const sa_segment* segs, int nseg, int N, int block, sa_layout** out);
+SA_API sa_status sa_build_layout(const sa_segment* segs, int nseg, int N, int block, sa_layout** out);
 
 /* nB blocks, n_pin / n_drop / n_cand (= C, sparsifiable) blocks, and cap =
  * nB - n_drop, the capacity an idx row needs.  Any output pointer may be NULL. */
-sa_status sa_layout_info(const sa_layout* L, int* nB, int* n_pin, int* n_drop, int* n_cand, int* cap);
+SA_API sa_status sa_layout_info(const sa_layout* L, int* nB, int* n_pin, int* n_drop, int* n_cand, int* cap);
 
 /* Host copy of the per-block classes (sa_block_class), nB bytes. */
-sa_status sa_layout_classes(const sa_layout* L, uint8_t* cls_out, int nB);
+SA_API sa_status sa_layout_classes(const sa_layout* L, uint8_t* cls_out, int nB);
 
 /* Drops one reference; the layout is freed when the count reaches zero. */
-sa_status sa_layout_release(sa_layout* L);
+SA_API sa_status sa_layout_release(sa_layout* L);
 
 /* Budget in kept candidates per sparse row [SDN "selector": a fraction of the
  * sparsifiable candidates]: clamp(floor(density * C + 1e-4), 1, C). */
-int sa_budget(float density, int n_cand);
+SA_API int sa_budget(float density, int n_cand);
 
 /*
  * sa_select_blocks [SDN "selector" + "host sync" paragraphs].
@@ -149,7 +155,7 @@ int sa_budget(float density, int n_cand);
  *   ws:         device workspace of at least sa_workspace_size bytes,
  *               header zeroed once with sa_workspace_init.
  */
-sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void* K, int B, int H, int d,
+SA_API sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void* K, int B, int H, int d,
                            float density, const uint8_t* head_mask, int min_active,
                            int32_t* idx, int32_t* counts, float* scores_out,
                            void* ws, size_t ws_bytes, sa_stream_t stream);
@@ -167,7 +173,7 @@ sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void* K, int
  *     (q - key) % r == 0 for some query of block i, plus G globals as above.
  * density is used by RADIAL only.  No workspace needed.
  */
-sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H, float density,
+SA_API sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H, float density,
                           const uint8_t* head_mask, int min_active,
                           int32_t* idx, int32_t* counts, sa_stream_t stream);
 
@@ -183,14 +189,14 @@ sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H,
  *   softmax_scale: 0 means 1/sqrt(d).
  *   O: device bf16 [B][H][N][d], fully written.
  */
-sa_status sa_block_sparse_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+SA_API sa_status sa_block_sparse_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
                                     const int32_t* idx, const int32_t* counts, int cap,
                                     const uint8_t* head_mask, int min_active, float softmax_scale,
                                     void* O, void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* sa_dense_attention: the same kernel over every tile of every head (the
  * dense baseline the speedup is measured against). */
-sa_status sa_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+SA_API sa_status sa_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
                              float softmax_scale, void* O, void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /*
@@ -198,25 +204,25 @@ sa_status sa_dense_attention(const void* Q, const void* K, const void* V, int B,
  * asks].  The only call that reads device memory back: it synchronises
  * `stream`.  Any of the outputs may be NULL.
  */
-sa_status sa_density(const int32_t* counts, int B, int H, int nB, const uint8_t* head_mask,
+SA_API sa_status sa_density(const int32_t* counts, int B, int H, int nB, const uint8_t* head_mask,
                      double* over_active, double* over_all, sa_stats* stats,
                      void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* Workspace bytes needed by every call for these sizes (selection and
  * attention regions are disjoint, so one workspace serves both). */
-sa_status sa_workspace_size(int B, int H, int N, int d, size_t* bytes);
+SA_API sa_status sa_workspace_size(int B, int H, int N, int d, size_t* bytes);
 
 /* Zeroes the workspace header (the sticky error word); enqueued on stream. */
-sa_status sa_workspace_init(void* ws, size_t ws_bytes, sa_stream_t stream);
+SA_API sa_status sa_workspace_init(void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /* Synchronises `stream`, reads and clears the workspace error word, and
  * returns SA_OK or the first device-side error recorded. */
-sa_status sa_check(void* ws, sa_stream_t stream);
+SA_API sa_status sa_check(void* ws, sa_stream_t stream);
 
-const char* sa_status_string(sa_status s);
+SA_API const char* sa_status_string(sa_status s);
 
 /* Library version string. */
-const char* sa_version(void);
+SA_API const char* sa_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,372 @@
+// C ABI entry points: argument validation, the layout cache, workspace
+// sizing, device-error readback and status strings.  Every entry point
+// validates before launching anything; hot calls never allocate or sync.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "sa_common.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+WsLayout ws_layout(int B, int H, int N, int d) {
+  WsLayout w;
+  const size_t BH = static_cast<size_t>(B) * H, nB = static_cast<size_t>(N) / kBlock;
+  size_t off = 0;
+  w.header = off;
+  off += sizeof(WsHeader);
+  w.qbar = off;
+  off += align256(BH * nB * d * sizeof(float));
+  w.kbar = off;
+  off += align256(BH * nB * d * sizeof(float));
+  w.items = off;
+  off += align256(BH * nB * sizeof(int4));
+  w.head_items = off;
+  off += align256(BH * nB * sizeof(int4));
+  w.head_np = off;
+  off += align256(BH * sizeof(int));
+  w.ulist = off;
+  off += align256(BH * nB * nB * sizeof(int32_t));
+  w.total = off;
+  return w;
+}
+
+cudaError_t device_info(DeviceInfo* out) {
+  static DeviceInfo cache[64];
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 64 && cache[dev].id == dev) {
+    *out = cache[dev];
+    return cudaSuccess;
+  }
+  DeviceInfo di;
+  di.id = dev;
+  if ((e = cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&di.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&di.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) return e;
+  if (dev < 64) cache[dev] = di;
+  *out = di;
+  return cudaSuccess;
+}
+
+}  // namespace sa
+
+using namespace sa;
+
+namespace {
+
+std::mutex g_layout_mu;
+std::vector<sa_layout*> g_layouts;  // cache of live layouts
+
+sa_status check_device(DeviceInfo* di) {
+  if (device_info(di) != cudaSuccess) return SA_ERR_CUDA;
+  if (di->cc_major != 10) return SA_ERR_UNSUPPORTED;
+  return SA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Head mask -> bit set; checks H and the minimum number of active heads.
+sa_status head_bits_of(const uint8_t* mask, int H, int min_active, uint64_t* bits) {
+  if (H <= 0 || H > kMaxHeads) return SA_ERR_SHAPE;
+  if (min_active < 0) return SA_ERR_INVALID_ARG;
+  uint64_t b = 0;
+  int active = 0;
+  for (int h = 0; h < H; ++h)
+    if (!mask || mask[h]) {
+      b |= 1ull << h;
+      ++active;
+    }
+  if (active < min_active) return SA_ERR_HEAD_MASK;
+  *bits = b;
+  return SA_OK;
+}
+
+bool density_ok(float rho) { return std::isfinite(rho) && rho > 0.f && rho <= 1.f; }
+
+sa_status ws_ok(const void* ws, size_t ws_bytes, int B, int H, int N, int d) {
+  if (!ws) return SA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SA_ERR_WORKSPACE;
+  if (ws_bytes < ws_layout(B, H, N, d).total) return SA_ERR_WORKSPACE;
+  return SA_OK;
+}
+
+sa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* sa_version(void) { return "prompt_aware_head_b200 0.1 (sm_100a)"; }
+
+const char* sa_status_string(sa_status s) {
+  switch (s) {
+    case SA_OK: return "ok";
+    case SA_ERR_INVALID_ARG: return "invalid argument";
+    case SA_ERR_SHAPE: return "unsupported shape";
+    case SA_ERR_LAYOUT: return "segments do not tile the sequence";
+    case SA_ERR_HEAD_MASK: return "fewer active heads than the minimum";
+    case SA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SA_ERR_BAD_INDEX: return "block index out of range or count above capacity";
+    case SA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case SA_ERR_UNSUPPORTED: return "device is not sm_100 (B200 class)";
+    case SA_ERR_CUDA: return "CUDA runtime error";
+  }
+  return "unknown status";
+}
+
+int sa_budget(float density, int n_cand) {
+  if (n_cand <= 0) return 0;
+  long k = static_cast<long>(std::floor(static_cast<double>(density) * n_cand + 1e-4));
+  if (k < 1) k = 1;
+  if (k > n_cand) k = n_cand;
+  return static_cast<int>(k);
+}
+
+sa_status sa_build_layout(const sa_segment* segs, int nseg, int N, int block, sa_layout** out) {
+  if (!out || nseg < 0 || (nseg > 0 && !segs)) return SA_ERR_INVALID_ARG;
+  if (block != kBlock || N <= 0 || N % block != 0 || N / block > kMaxBlocks) return SA_ERR_SHAPE;
+  // segments must tile [0, N) in order with known kinds
+  int pos = 0;
+  for (int s = 0; s < nseg; ++s) {
+    if (segs[s].kind < SA_SEG_TEXT || segs[s].kind > SA_SEG_OTHER || segs[s].start != pos || segs[s].len <= 0 ||
+        segs[s].len > N - pos)
+      return SA_ERR_LAYOUT;
+    pos += segs[s].len;
+  }
+  if (nseg > 0 && pos != N) return SA_ERR_LAYOUT;
+  DeviceInfo di;
+  sa_status st = check_device(&di);
+  if (st != SA_OK) return st;
+
+  std::lock_guard<std::mutex> lock(g_layout_mu);
+  for (sa_layout* L : g_layouts) {
+    if (L->N == N && L->block == block && L->device == di.id && static_cast<int>(L->segs.size()) == nseg &&
+        (nseg == 0 || std::memcmp(L->segs.data(), segs, sizeof(sa_segment) * nseg) == 0)) {
+      ++L->refcount;
+      *out = L;
+      return SA_OK;
+    }
+  }
+  sa_layout* L = new sa_layout();
+  L->N = N;
+  L->block = block;
+  L->nB = N / block;
+  L->segs.assign(segs, segs + nseg);
+  L->cls.assign(L->nB, static_cast<uint8_t>(kSparse));
+  // Per block: count image and padding tokens over the runs that overlap it.
+  for (int b = 0; b < L->nB; ++b) {
+    if (nseg == 0) break;
+    const int lo = b * block, hi = lo + block;
+    int img = 0, pad = 0;
+    for (int s = 0; s < nseg; ++s) {
+      const int a0 = std::max(lo, segs[s].start), a1 = std::min(hi, segs[s].start + segs[s].len);
+      if (a1 <= a0) continue;
+      if (segs[s].kind == SA_SEG_IMAGE) img += a1 - a0;
+      if (segs[s].kind == SA_SEG_PAD) pad += a1 - a0;
+    }
+    L->cls[b] = img == block ? kSparse : (pad == block ? kDrop : kPin);
+  }
+  std::vector<int32_t> rank(L->nB, -1);
+  int r = 0;
+  for (int b = 0; b < L->nB; ++b) {
+    if (L->cls[b] == kPin) ++L->n_pin;
+    if (L->cls[b] == kDrop) ++L->n_drop;
+    if (L->cls[b] == kSparse) rank[b] = r++;
+  }
+  L->n_cand = r;
+  L->cap = L->nB - L->n_drop;
+  L->device = di.id;
+  cudaError_t e = cudaMalloc(&L->d_cls, L->nB);
+  if (e == cudaSuccess) e = cudaMalloc(&L->d_sparse_rank, sizeof(int32_t) * L->nB);
+  if (e == cudaSuccess) e = cudaMemcpy(L->d_cls, L->cls.data(), L->nB, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(L->d_sparse_rank, rank.data(), sizeof(int32_t) * L->nB, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(L->d_cls);
+    cudaFree(L->d_sparse_rank);
+    delete L;
+    return SA_ERR_CUDA;
+  }
+  L->refcount = 1;
+  g_layouts.push_back(L);
+  *out = L;
+  return SA_OK;
+}
+
+sa_status sa_layout_info(const sa_layout* L, int* nB, int* n_pin, int* n_drop, int* n_cand, int* cap) {
+  if (!L) return SA_ERR_INVALID_ARG;
+  if (nB) *nB = L->nB;
+  if (n_pin) *n_pin = L->n_pin;
+  if (n_drop) *n_drop = L->n_drop;
+  if (n_cand) *n_cand = L->n_cand;
+  if (cap) *cap = L->cap;
+  return SA_OK;
+}
+
+sa_status sa_layout_classes(const sa_layout* L, uint8_t* cls_out, int nB) {
+  if (!L || !cls_out || nB != L->nB) return SA_ERR_INVALID_ARG;
+  std::memcpy(cls_out, L->cls.data(), L->nB);
+  return SA_OK;
+}
+
+sa_status sa_layout_release(sa_layout* L) {
+  if (!L) return SA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_layout_mu);
+  for (size_t i = 0; i < g_layouts.size(); ++i) {
+    if (g_layouts[i] != L) continue;
+    if (--L->refcount == 0) {
+      cudaFree(L->d_cls);
+      cudaFree(L->d_sparse_rank);
+      g_layouts.erase(g_layouts.begin() + i);
+      delete L;
+    }
+    return SA_OK;
+  }
+  return SA_ERR_INVALID_ARG;
+}
+
+sa_status sa_workspace_size(int B, int H, int N, int d, size_t* bytes) {
+  if (!bytes) return SA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || H > kMaxHeads || N <= 0 || N % kBlock || N / kBlock > kMaxBlocks || (d != 64 && d != 128))
+    return SA_ERR_SHAPE;
+  *bytes = ws_layout(B, H, N, d).total;
+  return SA_OK;
+}
+
+sa_status sa_workspace_init(void* ws, size_t ws_bytes, sa_stream_t stream) {
+  if (!ws || ws_bytes < sizeof(WsHeader)) return SA_ERR_WORKSPACE;
+  return from_cuda(cudaMemsetAsync(ws, 0, sizeof(WsHeader), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_check(void* ws, sa_stream_t stream) {
+  if (!ws) return SA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SA_ERR_CUDA;
+  int err = 0;
+  if (cudaMemcpy(&err, &static_cast<WsHeader*>(ws)->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SA_ERR_CUDA;
+  if (err && cudaMemset(&static_cast<WsHeader*>(ws)->err, 0, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
+  if (err & kErrBadIndex) return SA_ERR_BAD_INDEX;
+  if (err & kErrTimeout) return SA_ERR_TIMEOUT;
+  return SA_OK;
+}
+
+sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, float density,
+                           const uint8_t* head_mask, int min_active, int32_t* idx, int32_t* counts,
+                           float* scores_out, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  if (!L || !Q || !K || !idx || !counts) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K)) return SA_ERR_INVALID_ARG;
+  if (B <= 0 || (d != 64 && d != 128)) return SA_ERR_SHAPE;
+  if (static_cast<long long>(B) * H * L->N >= (1ll << 31)) return SA_ERR_SHAPE;
+  if (!density_ok(density)) return SA_ERR_INVALID_ARG;
+  uint64_t bits = 0;
+  sa_status st = head_bits_of(head_mask, H, min_active, &bits);
+  if (st != SA_OK) return st;
+  if ((st = ws_ok(ws, ws_bytes, B, H, L->N, d)) != SA_OK) return st;
+  DeviceInfo di;
+  if ((st = check_device(&di)) != SA_OK) return st;
+  if (di.id != L->device) return SA_ERR_INVALID_ARG;
+  const int k = sa_budget(density, L->n_cand);
+  return from_cuda(launch_select(L, Q, K, B, H, d, k, bits, idx, counts, scores_out, ws,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H, float density,
+                          const uint8_t* head_mask, int min_active, int32_t* idx, int32_t* counts,
+                          sa_stream_t stream) {
+  if (!L || !p || !idx || !counts) return SA_ERR_INVALID_ARG;
+  if (B <= 0) return SA_ERR_SHAPE;
+  if (p->kind < SA_PAT_RADIAL || p->kind > SA_PAT_DILATED) return SA_ERR_INVALID_ARG;
+  if (p->kind == SA_PAT_RADIAL && !density_ok(density)) return SA_ERR_INVALID_ARG;
+  if (p->kind != SA_PAT_RADIAL && (p->window_tokens < 0 || p->n_global_blocks < 0)) return SA_ERR_INVALID_ARG;
+  if (p->kind == SA_PAT_DILATED && p->dilation < 1) return SA_ERR_INVALID_ARG;
+  uint64_t bits = 0;
+  sa_status st = head_bits_of(head_mask, H, min_active, &bits);
+  if (st != SA_OK) return st;
+  DeviceInfo di;
+  if ((st = check_device(&di)) != SA_OK) return st;
+  if (di.id != L->device) return SA_ERR_INVALID_ARG;
+  const int k = p->kind == SA_PAT_RADIAL ? sa_budget(density, L->n_cand) : 0;
+  return from_cuda(launch_pattern(L, p->kind, p->window_tokens, p->n_global_blocks,
+                                  p->kind == SA_PAT_DILATED ? p->dilation : 1, k, B, H, bits, idx, counts,
+                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static sa_status attention_args_ok(const void* Q, const void* K, const void* V, const void* O, int B, int H, int N,
+                                   int d, float* scale) {
+  if (!Q || !K || !V || !O) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || H > kMaxHeads || (d != 64 && d != 128)) return SA_ERR_SHAPE;
+  if (N <= 0 || N % kBlock || N / kBlock > kMaxBlocks) return SA_ERR_SHAPE;
+  if (static_cast<long long>(B) * H * N >= (1ll << 31)) return SA_ERR_SHAPE;
+  if (!std::isfinite(*scale) || *scale < 0.f) return SA_ERR_INVALID_ARG;
+  if (*scale == 0.f) *scale = 1.0f / std::sqrt(static_cast<float>(d));
+  return SA_OK;
+}
+
+sa_status sa_block_sparse_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                    const int32_t* idx, const int32_t* counts, int cap, const uint8_t* head_mask,
+                                    int min_active, float softmax_scale, void* O, void* ws, size_t ws_bytes,
+                                    sa_stream_t stream) {
+  sa_status st = attention_args_ok(Q, K, V, O, B, H, N, d, &softmax_scale);
+  if (st != SA_OK) return st;
+  if (!idx || !counts) return SA_ERR_INVALID_ARG;
+  if (cap < 1 || cap > N / kBlock) return SA_ERR_SHAPE;
+  uint64_t bits = 0;
+  if ((st = head_bits_of(head_mask, H, min_active, &bits)) != SA_OK) return st;
+  if ((st = ws_ok(ws, ws_bytes, B, H, N, d)) != SA_OK) return st;
+  DeviceInfo di;
+  if ((st = check_device(&di)) != SA_OK) return st;
+  return from_cuda(launch_sparse_attention(Q, K, V, B, H, N, d, idx, counts, cap, bits, softmax_scale, O, ws,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                             float softmax_scale, void* O, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  sa_status st = attention_args_ok(Q, K, V, O, B, H, N, d, &softmax_scale);
+  if (st != SA_OK) return st;
+  if (!ws || !aligned16(ws) || ws_bytes < sizeof(WsHeader)) return SA_ERR_WORKSPACE;
+  DeviceInfo di;
+  if ((st = check_device(&di)) != SA_OK) return st;
+  return from_cuda(launch_dense_attention(Q, K, V, B, H, N, d, softmax_scale, O, ws,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_density(const int32_t* counts, int B, int H, int nB, const uint8_t* head_mask, double* over_active,
+                     double* over_all, sa_stats* stats, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  if (!counts) return SA_ERR_INVALID_ARG;
+  if (B <= 0 || nB <= 0 || nB > kMaxBlocks) return SA_ERR_SHAPE;
+  uint64_t bits = 0;
+  sa_status st = head_bits_of(head_mask, H, 0, &bits);
+  if (st != SA_OK) return st;
+  if (!ws || !aligned16(ws) || ws_bytes < sizeof(WsHeader)) return SA_ERR_WORKSPACE;
+  DeviceInfo di;
+  if ((st = check_device(&di)) != SA_OK) return st;
+  unsigned long long tiles = 0;
+  if (launch_density(counts, B, H, nB, bits, ws, &tiles, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SA_ERR_CUDA;
+  const int active = __builtin_popcountll(bits);
+  const double cells = static_cast<double>(nB) * nB;
+  const double da = active ? static_cast<double>(tiles) / (static_cast<double>(B) * active * cells) : 0.0;
+  const double dall = static_cast<double>(tiles) / (static_cast<double>(B) * H * cells);
+  if (over_active) *over_active = da;
+  if (over_all) *over_all = dall;
+  if (stats) {
+    stats->density_over_active = da;
+    stats->density_over_all = dall;
+    stats->tiles = static_cast<int64_t>(tiles);
+    stats->heads_active = active;
+  }
+  return SA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// Host-side internals shared by the C ABI (api.cpp) and the kernel launchers.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/sa.h"
+
+struct sa_layout {
+  int N = 0, block = 64, nB = 0;
+  int n_pin = 0, n_drop = 0, n_cand = 0, cap = 0;
+  std::vector<sa_segment> segs;
+  std::vector<uint8_t> cls;         // host copy of the block classes
+  int device = -1;
+  uint8_t* d_cls = nullptr;         // device [nB] block classes
+  int32_t* d_sparse_rank = nullptr; // device [nB]: index among SPARSE blocks, -1 otherwise
+  int refcount = 0;
+};
+
+namespace sa {
+
+// Workspace layout (byte offsets from the caller's workspace base).
+struct WsLayout {
+  size_t header = 0;        // WsHeader (256 B)
+  size_t qbar = 0, kbar = 0;  // fp32 [BH][nB][d] block means
+  size_t items = 0;         // int4 [BH*nB] attention work items (execution order)
+  size_t head_items = 0;    // int4 [BH][nB] per-head items before compaction
+  size_t head_np = 0;       // int32 [BH] items per head
+  size_t ulist = 0;         // int32 [BH][nB][nB] union lists (j | bits << 16)
+  size_t total = 0;
+};
+WsLayout ws_layout(int B, int H, int N, int d);
+
+struct DeviceInfo {
+  int id = -1, sm_count = 0, cc_major = 0, cc_minor = 0;
+};
+cudaError_t device_info(DeviceInfo* out);
+
+// Selection / pattern / density launchers (select.cu).
+cudaError_t launch_select(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, int k,
+                          uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out, void* ws,
+                          cudaStream_t s);
+// kind: 0 radial, 1 window+global, 2 dilated, 3 dense (every non-drop block).
+cudaError_t launch_pattern(const sa_layout* L, int kind, int W, int G, int r, int k, int B, int H,
+                           uint64_t head_bits, int32_t* idx, int32_t* counts, cudaStream_t s);
+cudaError_t launch_density(const int32_t* counts, int B, int H, int nB, uint64_t head_bits, void* ws,
+                           unsigned long long* host_tiles, cudaStream_t s);
+
+// Attention launchers (attention.cu).
+cudaError_t launch_sparse_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                    const int32_t* idx, const int32_t* counts, int cap, uint64_t head_bits,
+                                    float scale, void* O, void* ws, cudaStream_t s);
+cudaError_t launch_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                   float scale, void* O, void* ws, cudaStream_t s);
+
+}  // namespace sa
