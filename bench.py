@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of block-sparse attention driven by a per-input mask on B200.
+
+One step = the whole hot path over one batch of synthetic input already in
+HBM: block selection (pool, score, rank-select with pins/drops and head
+skipping), the attention work plan, and flash attention over the selected
+tiles.  Metric: effective TFLOP/s = 4 * 64 * 64 * d * (selected tiles) / step
+time, i.e. 4*B*H_active*N^2*d*density / t.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload joint|sdxl|video|stack|tiny]
+  python bench.py --impl reference ...     # the fp64 CPU oracle on a bounded sample
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own
+independent batch (seed = rank); value = all ranks' flops / max-over-ranks
+time (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, head_mask_for_layer, make_qkv  # noqa: E402
+
+METRIC = "effective TFLOP/s of block-sparse attention; speedup vs dense at 30% density"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def describe(w, rho):
+    segs = ", ".join("%s[%d,%d)" % ({0: "text", 1: "pad", 2: "image", 3: "other"}[k], s, s + l) for k, s, l in w.segments)
+    return "%s: B%d H%d d%d N%d%s, density %.2f%s" % (
+        w.name, w.B, w.H, w.d, w.N, (" (" + segs + ")") if segs else "", rho,
+        (", head mask %d of %d" % (int(head_mask_for_layer(w).sum()), w.H)) if w.head_mask or w.mask_runs else "")
+
+
+# ------------------------------------------------------------------ oracle (CPU) sample
+def oracle_sample(w, rho, target_s=8.0, seed=0):
+    """Times the fp64 oracle on one head: its full selection plus attention for
+    an evenly spaced subset of its query rows sized for about target_s."""
+    import oracle
+    mask = head_mask_for_layer(w)
+    h = int(np.flatnonzero(mask)[0])
+    Q, K, V = make_qkv(w, seed=seed, heads=[h])
+    Q, K, V = Q[:1], K[:1], V[:1]
+    t0 = time.perf_counter()
+    cls = oracle.layout(list(w.segments), w.N)
+    sc = oracle.scores(oracle.pool(Q), oracle.pool(K)).reshape(-1, w.nB, w.nB)
+    idx, cnt = oracle.select(sc, cls, 1, rho)
+    t_sel = time.perf_counter() - t0
+
+    def run(nrows):
+        rows = np.unique(np.linspace(0, w.N - 1, nrows).astype(np.int64))
+        t = time.perf_counter()
+        oracle.attention(Q, K, V, 1, idx, cnt, rows=rows)
+        return rows, time.perf_counter() - t
+
+    rows, t = run(256)
+    n = int(min(w.N, max(256, 256 * max(target_s - t_sel, 1.0) / max(t, 1e-6))))
+    rows, t_att = run(n)
+    flops = float(np.sum(4.0 * w.d * 64 * cnt[0, rows // 64]))
+    t_total = t_att + t_sel * len(rows) / w.N
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return {
+        "value": flops / t_total / 1e12,
+        "unit": UNIT,
+        "cores": cores,
+        "kind": "oracle",
+        "sample": "head %d of the workload: full fp64 selection for the head (%.2f s, charged pro rata) + fp64 "
+                  "attention for %d evenly spaced query rows (%.2f s)" % (h, t_sel, len(rows), t_att),
+        "seconds": t_total,
+    }
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_%d.csv" % os.getpid())
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8 or (self.uuid and self.uuid not in parts[0]):
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ traffic from the committed ncu summary
+def traffic_from_profile(kernel_src):
+    """dram bytes per launch recorded under profiles/ for the attention kernel, if
+    the kernel source has not changed since the capture (else None)."""
+    p = os.path.join(ROOT, "profiles", "sparse_attn_kernel_joint.md")
+    if not os.path.exists(p):
+        return None
+    digest = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(p):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("attention.cu sha256[:16]") != digest:
+        return None
+    try:
+        return float(vals["dram bytes per launch (full size)"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    import prompt_aware_head_b200 as sa
+
+    w = WORKLOADS[args.workload]
+    rho = args.density if args.density else w.densities[0]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    mask = head_mask_for_layer(w)
+    Qh, Kh, Vh = make_qkv(w, seed=rank)
+    pin = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (Qh, Kh, Vh)]
+    Q, K, V = (p.to(dev, non_blocking=False) for p in pin)
+    L = sa.Layout(list(w.segments), N)
+    ws_bytes = sa.sa_workspace_size(B, H, N, d)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    idx = torch.zeros((B, H, w.nB, L.cap), dtype=torch.int32, device=dev)
+    counts = torch.zeros((B, H, w.nB), dtype=torch.int32, device=dev)
+    O = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    O_host = torch.empty(O.shape, dtype=torch.bfloat16).pin_memory()
+    stream = torch.cuda.current_stream(dev)
+    sa.sa_workspace_init(ws, ws_bytes, stream)
+    in_bytes = 3 * Q.numel() * 2
+    flush = in_bytes < 2 * L2_BYTES
+    scratch = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev) if flush else None
+    k_budget = sa.sa_budget(rho, L.n_cand)
+    dense_short = k_budget >= L.n_cand
+    n_masked = int(H - mask.sum())
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        sa.sa_select_blocks(L, Q, K, B, H, d, rho, mask, w.min_active, idx, counts, None, ws, ws_bytes, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        sa.sa_attention_plan(idx, counts, B, H, N, d, L.cap, mask, w.min_active, ws, ws_bytes, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        sa.sa_attention_run(Q, K, V, B, H, N, d, mask, w.min_active, 0.0, O, ws, ws_bytes, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    launches_per_step = (1 if dense_short else 2) + 2 + 1 + (1 if n_masked else 0)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert sa.sa_check(ws, stream) == sa.SA_OK
+    _, _, st = sa.sa_density(counts, B, H, w.nB, mask, ws, ws_bytes, stream)
+    tiles = st.tiles
+    flops_step = 4.0 * 64 * 64 * d * tiles
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        if flush:
+            scratch.fill_(float(i))  # 512 MB write between steps, outside the per-step events
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    t_step = [e[0].elapsed_time(e[3]) for e in evs]
+    t_sel = [e[0].elapsed_time(e[1]) for e in evs]
+    t_plan = [e[1].elapsed_time(e[2]) for e in evs]
+    t_att = [e[2].elapsed_time(e[3]) for e in evs]
+    ms_step = statistics.mean(t_step)
+    ms_max = ms_step
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    value = world * flops_step / (ms_max * 1e-3) / 1e12
+    assert sa.sa_check(ws, stream) == sa.SA_OK
+
+    # dense baseline (same library, all heads, same inputs), and torch SDPA
+    dense_ms = sdpa_ms = None
+    if not args.no_dense:
+        Od = torch.empty_like(O)
+        for _ in range(3):
+            sa.sa_dense_attention(Q, K, V, B, H, N, d, 0.0, Od, ws, ws_bytes, stream)
+        de = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+        for a, b in de:
+            if flush:
+                scratch.fill_(1.0)
+            a.record(stream)
+            sa.sa_dense_attention(Q, K, V, B, H, N, d, 0.0, Od, ws, ws_bytes, stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = statistics.mean(a.elapsed_time(b) for a, b in de)
+        try:
+            f = torch.nn.functional.scaled_dot_product_attention
+            for _ in range(2):
+                f(Q, K, V)
+            se = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(3)]
+            for a, b in se:
+                a.record(stream)
+                f(Q, K, V)
+                b.record(stream)
+            torch.cuda.synchronize()
+            sdpa_ms = statistics.mean(a.elapsed_time(b) for a, b in se)
+        except Exception:
+            sdpa_ms = None
+        del Od
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e_steps = max(1, min(args.steps, 10))
+    ee = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    torch.cuda.synchronize()
+    ee[0].record(stream)
+    for _ in range(e2e_steps):
+        Q.copy_(pin[0], non_blocking=True)
+        K.copy_(pin[1], non_blocking=True)
+        V.copy_(pin[2], non_blocking=True)
+        sa.sa_select_blocks(L, Q, K, B, H, d, rho, mask, w.min_active, idx, counts, None, ws, ws_bytes, stream)
+        sa.sa_block_sparse_attention(Q, K, V, B, H, N, d, idx, counts, L.cap, mask, w.min_active, 0.0, O, ws,
+                                     ws_bytes, stream)
+        O_host.copy_(O, non_blocking=True)
+    ee[1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ee[0].elapsed_time(ee[1]) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    pk, pk_kind = peaks()
+    att_ms = statistics.mean(t_att)
+    sel_ms = statistics.mean(t_sel)
+    achieved = flops_step / (att_ms * 1e-3) / 1e12
+    traffic = traffic_from_profile(os.path.join(ROOT, "prompt_aware_head_b200", "csrc", "attention.cu"))
+    n_act = int(mask.sum())
+    sel_bytes = 2.0 * B * n_act * N * d * 2 + 4.0 * tiles + 4.0 * B * n_act * w.nB
+    sel_gbs = sel_bytes / (sel_ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; Q/K rank-8 sinusoidal position structure + noise, V ~ N(0,1); no weights)",
+        "config": {
+            "workload": describe(w, rho),
+            "B": B, "H": H, "N": N, "d": d, "density_budget": rho,
+            "density_realized": round(tiles / (B * n_act * w.nB ** 2), 5),
+            "selected_tiles": int(tiles),
+            "l2": "flushed between steps (512 MB write outside the per-step events)" if flush
+                  else "inputs larger than L2 (%.0f MB of Q/K/V)" % (in_bytes / 1e6),
+            "parallelism": "replicas x%d (independent batches, no collective)" % world,
+        },
+        "breakdown_ms": {"select": round(sel_ms, 5), "plan": round(statistics.mean(t_plan), 5),
+                         "attention": round(att_ms, 5)},
+        "speedup_vs_dense": round(dense_ms / ms_step, 3) if dense_ms else None,
+        "attention_speedup_vs_dense": round(dense_ms / att_ms, 3) if dense_ms else None,
+        "dense_ms": round(dense_ms, 5) if dense_ms else None,
+        "dense_tflops": round(4.0 * B * H * N * N * d / (dense_ms * 1e-3) / 1e12, 2) if dense_ms else None,
+        "torch_sdpa_dense_ms": round(sdpa_ms, 5) if sdpa_ms else None,
+        "speedup_vs_torch_sdpa": round(sdpa_ms / ms_step, 3) if sdpa_ms else None,
+        "roofline": {
+            "kernel": "sparse_attn_kernel<%d>" % d,
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": pk["bf16_tflops"],
+            "unit": "TFLOP/s",
+            "frac": round(achieved / pk["bf16_tflops"], 4),
+            "peak_kind": "%s burst dense bf16 (frac vs %s sustained %.1f: %.4f)" % (
+                pk_kind, pk_kind, pk["bf16_tflops_sustained"], achieved / pk["bf16_tflops_sustained"]),
+            "traffic": traffic,
+        },
+        "selection_roofline": {
+            "bound": "hbm", "achieved": round(sel_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(sel_gbs / pk["hbm_gbs"], 4), "algorithmic_bytes": int(sel_bytes),
+        },
+        "e2e": {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+                "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(O.numel() * 2),
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample(w, rho, target_s=args.cpu_seconds, seed=rank)
+        cb.pop("seconds", None)
+        out["cpu_baseline"] = cb
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_reference(args):
+    """The fp64 CPU oracle as it stands, timed on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    rho = args.density if args.density else w.densities[0]
+    per_step = max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, rho, target_s=min(per_step, 3.0))
+    vals, secs, last = [], [], None
+    for _ in range(args.steps):
+        last = oracle_sample(w, rho, target_s=per_step)
+        vals.append(last["value"])
+        secs.append(last["seconds"])
+    value = statistics.mean(vals)
+    out = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(secs), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded generator)",
+        "config": {"workload": describe(w, rho), "B": w.B, "H": w.H, "N": w.N, "d": w.d, "density_budget": rho},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last["cores"], "kind": "oracle",
+                         "sample": last["sample"]},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="joint")
+    ap.add_argument("--density", type=float, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -194,6 +194,22 @@ SA_API sa_status sa_block_sparse_attention(const void* Q, const void* K, const v
                                     const uint8_t* head_mask, int min_active, float softmax_scale,
                                     void* O, void* ws, size_t ws_bytes, sa_stream_t stream);
 
+/*
+ * The two halves of sa_block_sparse_attention, for callers that reuse one
+ * block list across calls or time the parts separately.
+ * sa_attention_plan reads (idx, counts) and writes the work plan into the
+ * workspace: the pairing of query blocks into 128-row tiles, the sorted
+ * union of each pair's lists with membership bits, and the longest-first
+ * work order.  sa_attention_run computes O from Q, K, V and the plan last
+ * written to the same workspace (same B, H, N, d and head mask).
+ */
+SA_API sa_status sa_attention_plan(const int32_t* idx, const int32_t* counts, int B, int H, int N, int d, int cap,
+                                   const uint8_t* head_mask, int min_active, void* ws, size_t ws_bytes,
+                                   sa_stream_t stream);
+SA_API sa_status sa_attention_run(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                  const uint8_t* head_mask, int min_active, float softmax_scale, void* O, void* ws,
+                                  size_t ws_bytes, sa_stream_t stream);
+
 /* sa_dense_attention: the same kernel over every tile of every head (the
  * dense baseline the speedup is measured against). */
 SA_API sa_status sa_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
@@ -220,6 +236,13 @@ SA_API sa_status sa_workspace_init(void* ws, size_t ws_bytes, sa_stream_t stream
 SA_API sa_status sa_check(void* ws, sa_stream_t stream);
 
 SA_API const char* sa_status_string(sa_status s);
+
+/* Diagnostic: out[i] = 2^y[i] computed by the polynomial exponential the
+ * attention softmax uses for part of its exponentials (round-to-nearest range
+ * reduction, degree-3 minimax polynomial on [-0.5, 0.5], relative error below
+ * 1e-4 for y >= -125; results for y < -125 are 2^-125).  Device arrays of n
+ * floats.  Not on the hot path; for tests. */
+SA_API sa_status sa_debug_exp2(const float* y, float* out, int n, sa_stream_t stream);
 
 /* Library version string. */
 SA_API const char* sa_version(void);

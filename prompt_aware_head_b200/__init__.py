@@ -64,12 +64,15 @@ _SIGS = {
     "sa_select_blocks": ([_P, _P, _P, _I, _I, _I, _F, _P, _I, _P, _P, _P, _P, _SZ, _P], _I),
     "sa_pattern_mask": ([_P, ctypes.POINTER(sa_pattern), _I, _I, _F, _P, _I, _P, _P, _P], _I),
     "sa_block_sparse_attention": ([_P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _F, _P, _P, _SZ, _P], _I),
+    "sa_attention_plan": ([_P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _SZ, _P], _I),
+    "sa_attention_run": ([_P, _P, _P, _I, _I, _I, _I, _P, _I, _F, _P, _P, _SZ, _P], _I),
     "sa_dense_attention": ([_P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _SZ, _P], _I),
     "sa_density": ([_P, _I, _I, _I, _P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
                     ctypes.POINTER(sa_stats), _P, _SZ, _P], _I),
     "sa_workspace_size": ([_I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "sa_workspace_init": ([_P, _SZ, _P], _I),
     "sa_check": ([_P, _P], _I),
+    "sa_debug_exp2": ([_P, _P, _I, _P], _I),
     "sa_status_string": ([_I], ctypes.c_char_p),
     "sa_version": ([], ctypes.c_char_p),
 }
@@ -196,6 +199,21 @@ def sa_block_sparse_attention(Q, K, V, B: int, H: int, N: int, d: int, idx, coun
                                           ws_bytes, _stream(stream)), "sa_block_sparse_attention")
 
 
+def sa_attention_plan(idx, counts, B: int, H: int, N: int, d: int, cap: int, head_mask, min_active: int, ws,
+                      ws_bytes: int, stream=None) -> None:
+    mptr, _keep = _host_mask(head_mask)
+    _check(_lib.sa_attention_plan(_addr(idx), _addr(counts), B, H, N, d, cap, mptr, min_active, _addr(ws), ws_bytes,
+                                  _stream(stream)), "sa_attention_plan")
+
+
+def sa_attention_run(Q, K, V, B: int, H: int, N: int, d: int, head_mask, min_active: int, softmax_scale: float, O,
+                     ws, ws_bytes: int, stream=None) -> None:
+    mptr, _keep = _host_mask(head_mask)
+    _check(_lib.sa_attention_run(_addr(Q), _addr(K), _addr(V), B, H, N, d, mptr, min_active,
+                                 ctypes.c_float(softmax_scale), _addr(O), _addr(ws), ws_bytes, _stream(stream)),
+           "sa_attention_run")
+
+
 def sa_dense_attention(Q, K, V, B: int, H: int, N: int, d: int, softmax_scale: float, O, ws, ws_bytes: int,
                        stream=None) -> None:
     _check(_lib.sa_dense_attention(_addr(Q), _addr(K), _addr(V), B, H, N, d, ctypes.c_float(softmax_scale),
@@ -209,6 +227,10 @@ def sa_density(counts, B: int, H: int, nB: int, head_mask, ws, ws_bytes: int, st
     _check(_lib.sa_density(_addr(counts), B, H, nB, mptr, ctypes.byref(a), ctypes.byref(b), ctypes.byref(st),
                            _addr(ws), ws_bytes, _stream(stream)), "sa_density")
     return a.value, b.value, st
+
+
+def sa_debug_exp2(y, out, n: int, stream=None) -> None:
+    _check(_lib.sa_debug_exp2(_addr(y), _addr(out), n, _stream(stream)), "sa_debug_exp2")
 
 
 def sa_status_string(status: int) -> str:

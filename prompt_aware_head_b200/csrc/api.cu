@@ -26,12 +26,14 @@ WsLayout ws_layout(int B, int H, int N, int d) {
   off += align256(BH * nB * d * sizeof(float));
   w.items = off;
   off += align256(BH * nB * sizeof(int4));
-  w.head_items = off;
-  off += align256(BH * nB * sizeof(int4));
-  w.head_np = off;
-  off += align256(BH * sizeof(int));
   w.ulist = off;
   off += align256(BH * nB * nB * sizeof(int32_t));
+  w.rowbits = off;
+  off += align256(BH * nB * (kMaxBlocks / 32) * sizeof(uint32_t));
+  w.lens = off;
+  off += align256(BH * nB * sizeof(int32_t));
+  w.totals = off;
+  off += align256(BH * 3 * sizeof(int32_t));
   w.total = off;
   return w;
 }
@@ -313,21 +315,44 @@ static sa_status attention_args_ok(const void* Q, const void* K, const void* V, 
   return SA_OK;
 }
 
+sa_status sa_attention_plan(const int32_t* idx, const int32_t* counts, int B, int H, int N, int d, int cap,
+                            const uint8_t* head_mask, int min_active, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  if (!idx || !counts) return SA_ERR_INVALID_ARG;
+  if (B <= 0 || (d != 64 && d != 128) || N <= 0 || N % kBlock || N / kBlock > kMaxBlocks) return SA_ERR_SHAPE;
+  if (cap < 1 || cap > N / kBlock) return SA_ERR_SHAPE;
+  uint64_t bits = 0;
+  sa_status st = head_bits_of(head_mask, H, min_active, &bits);
+  if (st != SA_OK) return st;
+  if ((st = ws_ok(ws, ws_bytes, B, H, N, d)) != SA_OK) return st;
+  DeviceInfo di;
+  if ((st = check_device(&di)) != SA_OK) return st;
+  return from_cuda(launch_attention_plan(idx, counts, B, H, N, d, cap, bits, ws,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_attention_run(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                           const uint8_t* head_mask, int min_active, float softmax_scale, void* O, void* ws,
+                           size_t ws_bytes, sa_stream_t stream) {
+  sa_status st = attention_args_ok(Q, K, V, O, B, H, N, d, &softmax_scale);
+  if (st != SA_OK) return st;
+  uint64_t bits = 0;
+  if ((st = head_bits_of(head_mask, H, min_active, &bits)) != SA_OK) return st;
+  if ((st = ws_ok(ws, ws_bytes, B, H, N, d)) != SA_OK) return st;
+  DeviceInfo di;
+  if ((st = check_device(&di)) != SA_OK) return st;
+  return from_cuda(launch_attention_run(Q, K, V, B, H, N, d, bits, softmax_scale, O, ws,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 sa_status sa_block_sparse_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
                                     const int32_t* idx, const int32_t* counts, int cap, const uint8_t* head_mask,
                                     int min_active, float softmax_scale, void* O, void* ws, size_t ws_bytes,
                                     sa_stream_t stream) {
   sa_status st = attention_args_ok(Q, K, V, O, B, H, N, d, &softmax_scale);
   if (st != SA_OK) return st;
-  if (!idx || !counts) return SA_ERR_INVALID_ARG;
-  if (cap < 1 || cap > N / kBlock) return SA_ERR_SHAPE;
-  uint64_t bits = 0;
-  if ((st = head_bits_of(head_mask, H, min_active, &bits)) != SA_OK) return st;
-  if ((st = ws_ok(ws, ws_bytes, B, H, N, d)) != SA_OK) return st;
-  DeviceInfo di;
-  if ((st = check_device(&di)) != SA_OK) return st;
-  return from_cuda(launch_sparse_attention(Q, K, V, B, H, N, d, idx, counts, cap, bits, softmax_scale, O, ws,
-                                           reinterpret_cast<cudaStream_t>(stream)));
+  if ((st = sa_attention_plan(idx, counts, B, H, N, d, cap, head_mask, min_active, ws, ws_bytes, stream)) != SA_OK)
+    return st;
+  return sa_attention_run(Q, K, V, B, H, N, d, head_mask, min_active, softmax_scale, O, ws, ws_bytes, stream);
 }
 
 sa_status sa_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
@@ -367,6 +392,14 @@ sa_status sa_density(const int32_t* counts, int B, int H, int nB, const uint8_t*
     stats->heads_active = active;
   }
   return SA_OK;
+}
+
+sa_status sa_debug_exp2(const float* y, float* out, int n, sa_stream_t stream) {
+  if (!y || !out || n < 0) return SA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  sa_status st = check_device(&di);
+  if (st != SA_OK) return st;
+  return from_cuda(launch_exp2_poly(y, out, n, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -53,7 +53,8 @@ struct AttnArgs {
 
 constexpr int kThreads = 192;
 constexpr int kNoBlock = 0xFFFF;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+constexpr float kRescaleThreshold = 8.0f;
+constexpr uint32_t kBackoffNs = 40;            // producer / MMA poll back-off  // log2 units: rescale O when the max grows by > 2^8
 
 struct Item {
   int bh, i0, i1, len, off;
@@ -168,18 +169,117 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint6
   }
 }
 
+// ---------------------------------------------------------------- softmax arithmetic
+// Packed fp32 pair operations (Blackwell f32x2 FMA-pipe instructions).
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                     float c1) {
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n mov.b64 rc, {%6, %7};\n"
+      " fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+__device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
+  asm("{\n .reg .b64 ra, rb;\n mov.b64 ra, {%0, %1};\n mov.b64 rb, {%2, %3};\n add.f32x2 ra, ra, rb;\n"
+      " mov.b64 {%0, %1}, ra;\n}\n"
+      : "+f"(s0), "+f"(s1)
+      : "f"(a0), "f"(a1));
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^y for a pair of values on the FMA pipe, to take load off the MUFU unit.
+// Range reduction y = j + f with j = round(y) (adding 1.5 * 2^23 leaves the
+// integer in the low mantissa bits) and f in [-0.5, 0.5]; 2^f by a degree-3
+// polynomial fitted here with the Remez exchange algorithm for minimax
+// relative error on [-0.5, 0.5] (max relative error 7.5e-5, far below the
+// bf16 resolution P is stored in); 2^j is added into the exponent field.
+// y is clamped at -125 so the exponent stays in the normal range.
+__device__ __forceinline__ void exp2_poly2(float y0, float y1, float& p0, float& p1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f, c2 = 0.2426111251115799f,
+                  c3 = 0.0551716685295105f;
+  y0 = fmaxf(y0, -125.f);
+  y1 = fmaxf(y1, -125.f);
+  float t0 = y0, t1 = y1;
+  add2(t0, t1, kMagic, kMagic);
+  float j0 = t0, j1 = t1;
+  add2(j0, j1, -kMagic, -kMagic);
+  float f0 = y0, f1 = y1;
+  add2(f0, f1, -j0, -j1);
+  float q0, q1;
+  fma2(q0, q1, f0, f1, c3, c3, c2, c2);
+  fma2(q0, q1, q0, q1, f0, f1, c1, c1);
+  fma2(q0, q1, q0, q1, f0, f1, c0, c0);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// One pass over 64 of a row's S values (raw fp32 bits, one key block):
+// p = 2^(x*c - m), packed to bf16 pairs in pk[0..32), accumulated into the
+// pair sums s[8]; the raw max is tracked into mv0/mv1 when kTrack is set.
+// One pair in four goes through the polynomial, the rest through MUFU ex2.
+template <bool kTrack>
+__device__ __forceinline__ void exp_half(const uint32_t* x, float c, float m, uint32_t* pk, float (&s)[8],
+                                         float& mv0, float& mv1) {
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const float x0 = __uint_as_float(x[2 * q]), x1 = __uint_as_float(x[2 * q + 1]);
+    if (kTrack) {
+      if (q & 1) mv1 = max3f(mv1, x0, x1);
+      else mv0 = max3f(mv0, x0, x1);
+    }
+    float y0, y1, p0, p1;
+    fma2(y0, y1, x0, x1, c, c, -m, -m);
+    if ((q & 3) == 0) {
+      exp2_poly2(y0, y1, p0, p1);
+    } else {
+      p0 = ex2(y0);
+      p1 = ex2(y1);
+    }
+    add2(s[2 * (q & 3)], s[2 * (q & 3) + 1], p0, p1);
+    pk[q] = pack_bf16x2(p0, p1);
+  }
+}
+
+__device__ __forceinline__ float sum8(const float (&s)[8]) {
+  return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+}
+
+__device__ __forceinline__ float row_max(const uint32_t (&x)[128], bool b0, bool b1) {
+  float mv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    if (!(ch < 2 ? b0 : b1)) continue;
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      mv[q & 3] = max3f(mv[q & 3], __uint_as_float(x[32 * ch + 2 * q]), __uint_as_float(x[32 * ch + 2 * q + 1]));
+  }
+  return fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3]));
+}
+
 // ---------------------------------------------------------------- kernel
 template <int D>
 struct AttnSmem {
-  static constexpr int kTile = 128 * D * 2;      // 128 rows x D bf16
+  static constexpr int kTile = 128 * D * 2;      // 128 rows x D bf16 (a Q tile, or a K / V pair)
   static constexpr int kChunk = 128 * 128;       // one 64-column chunk of a 128-row tile
-  static constexpr int kStages = (D == 128) ? 2 : 4;
+  // K and V live in separate rings: a K stage is free as soon as its S MMA
+  // completes, a V stage once its PV MMA does.  Three stages each cover the
+  // ~1 us latency of an L2-resident TMA load at d = 128 (224 KB in all).
+  static constexpr int kQBuf = (D == 128) ? 1 : 2;
+  static constexpr int kNK = (D == 128) ? 3 : 4;
+  static constexpr int kNV = (D == 128) ? 3 : 4;
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + 2 * kTile;
-  static constexpr int kV = kK + kStages * kTile;
-  static constexpr int kBar = kV + kStages * kTile;
-  static constexpr int kBytes = kBar + 1024;     // barriers + flags
+  static constexpr int kK = kQ + kQBuf * kTile;
+  static constexpr int kV = kK + kNK * kTile;
+  static constexpr int kBar = kV + kNV * kTile;
+  static constexpr int kBytes = kBar + 512;      // barriers + flags
   static constexpr int kAlloc = kBytes + 1024;   // slack for 1024-B alignment
+  static_assert(kAlloc <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
 };
 
 template <int D>
@@ -187,22 +287,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using S = AttnSmem<D>;
-  constexpr int NST = S::kStages;
+  constexpr int NK = S::kNK, NV = S::kNV, QB = S::kQBuf;
   constexpr uint32_t kTxBlock = 64 * D * 2;  // bytes of one 64-row block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + S::kBar);
-  uint64_t* q_full = bars + 0;              // [2]
-  uint64_t* q_empty = bars + 2;             // [2]
+  uint64_t* q_full = bars + 0;              // [QB]
+  uint64_t* q_empty = bars + 2;             // [QB] after the last S MMA of an item
   uint64_t* s_full = bars + 4;              // [2]
   uint64_t* p_full = bars + 6;              // [2]
   uint64_t* o_done = bars + 8;              // after every PV
   uint64_t* o_final = bars + 9;             // after the last PV of an item
   uint64_t* drain = bars + 10;              // abort path
-  uint64_t* k_full = bars + 12;             // [NST]
-  uint64_t* v_full = k_full + NST;          // [NST]
-  uint64_t* kv_empty = v_full + NST;        // [NST]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(kv_empty + NST);
+  uint64_t* k_full = bars + 12;             // [NK]
+  uint64_t* k_empty = k_full + NK;          // [NK] after the S MMA that read the stage
+  uint64_t* v_full = k_empty + NK;          // [NV]
+  uint64_t* v_empty = v_full + NV;          // [NV] after the PV MMA that read the stage
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(v_empty + NV);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -216,10 +317,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(o_done, 1);
     mbar_init(o_final, 1);
     mbar_init(drain, 1);
-    for (int i = 0; i < NST; ++i) {
+    for (int i = 0; i < NK; ++i) {
       mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < NV; ++i) {
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     *abort_flag = 0;
     mbar_fence_init();
@@ -239,9 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ======================= TMA producer =======================
     if (lane == 0) {
       uint32_t g = 0, t = 0;
-      int ld_phase[NST];
-      int q_phase[2] = {-1, -1};
-      for (int s = 0; s < NST; ++s) ld_phase[s] = -1;
+      int k_phase[NK], v_phase[NV], q_phase[2] = {-1, -1};
+      for (int i = 0; i < NK; ++i) k_phase[i] = -1;
+      for (int i = 0; i < NV; ++i) v_phase[i] = -1;
       bool ok = true;
       for (int r = 0; ok; ++r) {
         const int k = item_index(r, cta, G);
@@ -249,8 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = load_item(a, k);
         const int nsteps = (it.len + 1) >> 1;
         if (nsteps == 0) continue;
-        const int qb = t & 1;
-        if (t >= 2 && !mbar_wait(&q_empty[qb], ((t >> 1) - 1) & 1, abort_flag, a.err)) { ok = false; break; }
+        const int qb = t % QB;
+        const uint32_t uq = t / QB;
+        if (uq >= 1 && !mbar_wait(&q_empty[qb], (uq - 1) & 1, abort_flag, a.err, kBackoffNs)) { ok = false; break; }
         const int row0 = it.bh * a.N;
         uint8_t* qdst = sm + S::kQ + qb * S::kTile;
         mbar_expect_tx(&q_full[qb], (it.i1 != kNoBlock ? 2u : 1u) * kTxBlock);
@@ -259,41 +364,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(qdst + c * S::kChunk, &tmQ, 64 * c, row0 + 64 * it.i0, &q_full[qb]);
           if (it.i1 != kNoBlock) tma_load_2d(qdst + c * S::kChunk + 8192, &tmQ, 64 * c, row0 + 64 * it.i1, &q_full[qb]);
         }
-        q_phase[qb] = (t >> 1) & 1;
+        q_phase[qb] = uq & 1;
         for (int s = 0; s < nsteps; ++s, ++g) {
-          const int st = g % NST;
-          const uint32_t u = g / NST;
-          if (u >= 1 && !mbar_wait(&kv_empty[st], (u - 1) & 1, abort_flag, a.err)) { ok = false; break; }
           const uint32_t e0 = load_entry(a, it, 2 * s);
           const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
           const uint32_t e1 = nblk == 2 ? load_entry(a, it, 2 * s + 1) : 0u;
           const int j0 = e0 & 0xFFFF, j1 = e1 & 0xFFFF;
-          uint8_t* kdst = sm + S::kK + st * S::kTile;
-          uint8_t* vdst = sm + S::kV + st * S::kTile;
-          mbar_expect_tx(&k_full[st], nblk * kTxBlock);
+          const int kst = g % NK;
+          const uint32_t uk = g / NK;
+          if (uk >= 1 && !mbar_wait(&k_empty[kst], (uk - 1) & 1, abort_flag, a.err, kBackoffNs)) { ok = false; break; }
+          uint8_t* kdst = sm + S::kK + kst * S::kTile;
+          mbar_expect_tx(&k_full[kst], nblk * kTxBlock);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(kdst + c * S::kChunk, &tmK, 64 * c, row0 + 64 * j0, &k_full[st]);
-            if (nblk == 2) tma_load_2d(kdst + c * S::kChunk + 8192, &tmK, 64 * c, row0 + 64 * j1, &k_full[st]);
+            tma_load_2d(kdst + c * S::kChunk, &tmK, 64 * c, row0 + 64 * j0, &k_full[kst]);
+            if (nblk == 2) tma_load_2d(kdst + c * S::kChunk + 8192, &tmK, 64 * c, row0 + 64 * j1, &k_full[kst]);
           }
-          mbar_expect_tx(&v_full[st], nblk * kTxBlock);
+          k_phase[kst] = uk & 1;
+          const int vst = g % NV;
+          const uint32_t uv = g / NV;
+          if (uv >= 1 && !mbar_wait(&v_empty[vst], (uv - 1) & 1, abort_flag, a.err, kBackoffNs)) { ok = false; break; }
+          uint8_t* vdst = sm + S::kV + vst * S::kTile;
+          mbar_expect_tx(&v_full[vst], nblk * kTxBlock);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(vdst + c * S::kChunk, &tmV, 64 * c, row0 + 64 * j0, &v_full[st]);
-            if (nblk == 2) tma_load_2d(vdst + c * S::kChunk + 8192, &tmV, 64 * c, row0 + 64 * j1, &v_full[st]);
+            tma_load_2d(vdst + c * S::kChunk, &tmV, 64 * c, row0 + 64 * j0, &v_full[vst]);
+            if (nblk == 2) tma_load_2d(vdst + c * S::kChunk + 8192, &tmV, 64 * c, row0 + 64 * j1, &v_full[vst]);
           }
-          ld_phase[st] = u & 1;
+          v_phase[vst] = uv & 1;
         }
         ++t;
       }
       if (!ok || *abort_flag) {
         // Drain: let every load this thread issued land before the CTA exits.
-        for (int s = 0; s < NST; ++s)
-          if (ld_phase[s] >= 0) {
-            mbar_wait_drain(&k_full[s], ld_phase[s], a.err);
-            mbar_wait_drain(&v_full[s], ld_phase[s], a.err);
-          }
-        for (int b = 0; b < 2; ++b)
+        for (int i = 0; i < NK; ++i)
+          if (k_phase[i] >= 0) mbar_wait_drain(&k_full[i], k_phase[i], a.err);
+        for (int i = 0; i < NV; ++i)
+          if (v_phase[i] >= 0) mbar_wait_drain(&v_full[i], v_phase[i], a.err);
+        for (int b = 0; b < QB; ++b)
           if (q_phase[b] >= 0) mbar_wait_drain(&q_full[b], q_phase[b], a.err);
       }
     }
@@ -303,15 +411,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
       uint32_t g = 0, t = 0;
       bool ok = true, have_pend = false;
-      uint32_t pg = 0, pst = 0, pacc = 0, plast = 0;
+      uint32_t pg = 0, pacc = 0, plast = 0;
       int pnblk = 0;
       auto do_pv = [&]() -> bool {
-        if (!mbar_wait(&p_full[pg & 1], (pg >> 1) & 1, abort_flag, a.err)) return false;
-        if (!mbar_wait(&v_full[pst], (pg / NST) & 1, abort_flag, a.err)) return false;
+        const int vst = pg % NV;
+        if (!mbar_wait(&p_full[pg & 1], (pg >> 1) & 1, abort_flag, a.err, kBackoffNs)) return false;
+        if (!mbar_wait(&v_full[vst], (pg / NV) & 1, abort_flag, a.err, kBackoffNs)) return false;
         tc_fence_after();
-        const uint64_t bdesc = smem_desc_sw128(smem_u32(sm + S::kV + pst * S::kTile), S::kChunk, 1024);
+        const uint64_t bdesc = smem_desc_sw128(smem_u32(sm + S::kV + vst * S::kTile), S::kChunk, 1024);
         issue_pv(tm + 256, tm + (pg & 1) * 128, bdesc, idesc_pv, pacc, pnblk);
-        tc_commit(&kv_empty[pst]);
+        tc_commit(&v_empty[vst]);
         tc_commit(o_done);
         if (plast) tc_commit(o_final);
         return true;
@@ -322,22 +431,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = load_item(a, k);
         const int nsteps = (it.len + 1) >> 1;
         if (nsteps == 0) continue;
-        const int qb = t & 1;
-        if (!mbar_wait(&q_full[qb], (t >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
+        const int qb = t % QB;
+        if (!mbar_wait(&q_full[qb], (t / QB) & 1, abort_flag, a.err, kBackoffNs)) { ok = false; break; }
         const uint64_t adesc = smem_desc_sw128(smem_u32(sm + S::kQ + qb * S::kTile), 16, 1024);
         for (int s = 0; s < nsteps; ++s, ++g) {
-          const int st = g % NST;
-          if (!mbar_wait(&k_full[st], (g / NST) & 1, abort_flag, a.err)) { ok = false; break; }
+          const int kst = g % NK;
+          if (!mbar_wait(&k_full[kst], (g / NK) & 1, abort_flag, a.err, kBackoffNs)) { ok = false; break; }
           tc_fence_after();
           const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
-          const uint64_t bdesc = smem_desc_sw128(smem_u32(sm + S::kK + st * S::kTile), 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sm + S::kK + kst * S::kTile), 16, 1024);
           issue_qk<D>(tm + (g & 1) * 128, adesc, bdesc, idesc_bf16_f32(128, 64 * nblk, 0, 0));
           tc_commit(&s_full[g & 1]);
+          tc_commit(&k_empty[kst]);
           if (s == nsteps - 1) tc_commit(&q_empty[qb]);
           if (have_pend && !do_pv()) { ok = false; break; }
           have_pend = true;
           pg = g;
-          pst = st;
           pnblk = nblk;
           pacc = s > 0 ? 1u : 0u;
           plast = (s == nsteps - 1) ? 1u : 0u;
@@ -377,74 +486,96 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       float m = -INFINITY, l = 0.f;
+      // union entries are prefetched one step ahead (global loads off the critical path)
+      uint32_t e0n = load_entry(a, it, 0);
+      uint32_t e1n = it.len > 1 ? load_entry(a, it, 1) : 0u;
       for (int s = 0; s < nsteps; ++s, ++g) {
         const int sb = g & 1;
+        const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
+        const uint32_t e0 = e0n, e1 = nblk == 2 ? e1n : 0u;
+        if (2 * s + 2 < it.len) e0n = load_entry(a, it, 2 * s + 2);
+        if (2 * s + 3 < it.len) e1n = load_entry(a, it, 2 * s + 3);
         if (!warp_wait(&s_full[sb], (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
         tc_fence_after();
-        const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
-        const uint32_t e0 = load_entry(a, it, 2 * s);
-        const uint32_t e1 = nblk == 2 ? load_entry(a, it, 2 * s + 1) : 0u;
         const bool b0 = (e0 >> (16 + half)) & 1u;
         const bool b1 = (e1 >> (16 + half)) & 1u;
         const uint32_t s_col = t_lane + sb * 128;
         uint32_t x[128];
-        if (b0) {
-          tmem_ld32(s_col, x);
-          tmem_ld32(s_col + 32, x + 32);
-        }
-        if (b1) {
-          tmem_ld32(s_col + 64, x + 64);
-          tmem_ld32(s_col + 96, x + 96);
-        }
-        if (b0 || b1) tmem_wait_ld();
-        float mx = -INFINITY;
-        if (b0) {
-#pragma unroll
-          for (int q = 0; q < 64; ++q) mx = fmaxf(mx, __uint_as_float(x[q]));
-        }
-        if (b1) {
-#pragma unroll
-          for (int q = 64; q < 128; ++q) mx = fmaxf(mx, __uint_as_float(x[q]));
-        }
-        mx *= c;  // c > 0: max commutes with the scaling
-        const float m_new = fmaxf(m, mx);
-        float m_use = m, alpha = 1.f;
-        bool rescale = false;
-        if (m == -INFINITY) {
-          m_use = m_new;
-        } else if (m_new - m > kRescaleThreshold) {
-          m_use = m_new;
-          alpha = ex2(m - m_new);
-          rescale = true;
-        }
-        float sum = 0.f;
         uint32_t pk[64];
-        if (b0) {
+        float sv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float mv0 = -INFINITY, mv1 = -INFINITY;
+        float sum = 0.f, alpha = 1.f;
+        bool rescale = false;
+        if (!(b0 || b1)) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const float p0 = ex2(fmaf(__uint_as_float(x[2 * q]), c, -m_use));
-            const float p1 = ex2(fmaf(__uint_as_float(x[2 * q + 1]), c, -m_use));
-            sum += p0 + p1;
-            pk[q] = pack_bf16x2(p0, p1);
+          for (int q = 0; q < 64; ++q) pk[q] = 0u;
+        } else if (__any_sync(0xffffffffu, m == -INFINITY)) {
+          // first selected block of this half (warp-uniform): find the max first
+          if (b0) {
+            tmem_ld32(s_col, x);
+            tmem_ld32(s_col + 32, x + 32);
           }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 32; ++q) pk[q] = 0u;
-        }
-        if (b1) {
-#pragma unroll
-          for (int q = 32; q < 64; ++q) {
-            const float p0 = ex2(fmaf(__uint_as_float(x[2 * q]), c, -m_use));
-            const float p1 = ex2(fmaf(__uint_as_float(x[2 * q + 1]), c, -m_use));
-            sum += p0 + p1;
-            pk[q] = pack_bf16x2(p0, p1);
+          if (b1) {
+            tmem_ld32(s_col + 64, x + 64);
+            tmem_ld32(s_col + 96, x + 96);
           }
-        } else {
+          tmem_wait_ld();
+          const float m_new = fmaxf(m, row_max(x, b0, b1) * c);  // c > 0: max commutes with the scaling
+          rescale = m != -INFINITY && m_new > m;
+          alpha = rescale ? ex2(m - m_new) : 1.f;
+          m = m_new;
+          if (b0) exp_half<false>(x, c, m, pk, sv, mv0, mv1);
+          else {
 #pragma unroll
-          for (int q = 32; q < 64; ++q) pk[q] = 0u;
+            for (int q = 0; q < 32; ++q) pk[q] = 0u;
+          }
+          if (b1) exp_half<false>(x + 64, c, m, pk + 32, sv, mv0, mv1);
+          else {
+#pragma unroll
+            for (int q = 32; q < 64; ++q) pk[q] = 0u;
+          }
+          sum = sum8(sv);
+        } else {
+          // Fused pass with the running (possibly stale) max m; the first
+          // half's exponentials overlap the second half's TMEM load.  Only
+          // when a row's max grows by more than 2^8 is the pass redone with
+          // the new max and O rescaled.
+          if (b0) {
+            tmem_ld32(s_col, x);
+            tmem_ld32(s_col + 32, x + 32);
+            tmem_wait_ld();
+          }
+          if (b1) {
+            tmem_ld32(s_col + 64, x + 64);
+            tmem_ld32(s_col + 96, x + 96);
+          }
+          if (b0) exp_half<true>(x, c, m, pk, sv, mv0, mv1);
+          else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) pk[q] = 0u;
+          }
+          if (b1) {
+            tmem_wait_ld();
+            exp_half<true>(x + 64, c, m, pk + 32, sv, mv0, mv1);
+          } else {
+#pragma unroll
+            for (int q = 32; q < 64; ++q) pk[q] = 0u;
+          }
+          sum = sum8(sv);
+          const float mx = fmaxf(mv0, mv1) * c;
+          rescale = mx > m + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, rescale)) {
+            const float m_new = rescale ? mx : m;
+            alpha = rescale ? ex2(m - m_new) : 1.f;
+            m = m_new;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) sv[u] = 0.f;
+            if (b0) exp_half<false>(x, c, m, pk, sv, mv0, mv1);
+            if (b1) exp_half<false>(x + 64, c, m, pk + 32, sv, mv0, mv1);
+            sum = sum8(sv);
+          }
         }
         l = l * alpha + sum;
-        m = m_use;
         if (__any_sync(0xffffffffu, rescale)) {
           // O (TMEM) holds PV results up to step g-1: wait for PV_{g-1}, then scale.
           if (!warp_wait(o_done, (g - 1) & 1, abort_flag, a.err)) { ok = false; break; }
@@ -503,168 +634,162 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- planner
-// One CTA per head (b, h).  Picks the pairing stride s in {1, 2, 4} that
-// minimises the summed union length, builds every pair's sorted union list
-// with membership bits, and orders the pairs by union length (longest
-// first) for the persistent kernel.  Validates every block index.
-constexpr int kPlanThreads = 512;
+// Five small kernels, each parallel over (head, query block):
+//  1. rowbits: each query block's list as a bitmap over key blocks (validates
+//     every index and count);
+//  2. union sizes of the candidate pairs for strides 1, 2 and 4, summed per
+//     head;
+//  3. per head, the stride with the smallest summed union; each pair's sorted
+//     union list with membership bits;
+//  4. per head, pairs ordered by union length (longest first) by rank counting;
+//  5. concatenation of the per-head item lists.
+constexpr int kWords = kMaxBlocks / 32;  // bitmap words per row
+__device__ __forceinline__ int stride_of(int si) { return 1 << si; }  // pairing strides 1, 2, 4
 
-__device__ __forceinline__ int pair_partner(int a, int s, int nB) {
-  return (a + s < nB) ? a + s : -1;
+__device__ __forceinline__ int pair_partner(int a, int s, int nB) { return (a + s < nB) ? a + s : -1; }
+__device__ __forceinline__ bool pair_first(int a, int s) { return ((a / s) & 1) == 0; }
+
+__global__ void __launch_bounds__(256) plan_rowbits_kernel(const int32_t* __restrict__ idx,
+                                                           const int32_t* __restrict__ counts, int nB, int cap,
+                                                           int H, uint64_t head_bits, uint32_t* __restrict__ rowbits,
+                                                           int* __restrict__ totals, int* __restrict__ err) {
+  __shared__ uint32_t bm[8][kWords];
+  const int bh = blockIdx.y, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * 8 + w;
+  if (!((head_bits >> (bh % H)) & 1ull) || i >= nB) return;
+  if (i == 0 && lane < 3) totals[bh * 3 + lane] = 0;
+  const int nwords = (nB + 31) >> 5;
+  bm[w][lane] = 0u;
+  __syncwarp();
+  int cnt = counts[static_cast<size_t>(bh) * nB + i];
+  if (cnt > cap || cnt < 0) {
+    if (lane == 0) atomicOr(err, kErrBadIndex);
+    cnt = cnt < 0 ? 0 : cap;
+  }
+  const int32_t* lst = idx + (static_cast<size_t>(bh) * nB + i) * cap;
+  for (int e = lane; e < cnt; e += 32) {
+    const int j = lst[e];
+    if (j < 0 || j >= nB) {
+      atomicOr(err, kErrBadIndex);
+      continue;
+    }
+    atomicOr(&bm[w][j >> 5], 1u << (j & 31));
+  }
+  __syncwarp();
+  if (lane < nwords) rowbits[(static_cast<size_t>(bh) * nB + i) * kWords + lane] = bm[w][lane];
 }
 
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ idx,
-                                                            const int32_t* __restrict__ counts, int nB, int cap,
-                                                            int H, uint64_t head_bits, int4* __restrict__ head_items,
-                                                            int* __restrict__ head_np, int32_t* __restrict__ ulist,
-                                                            int* __restrict__ err) {
-  __shared__ uint32_t bm[kPlanThreads / 32][2][kMaxBlocks / 32];
-  __shared__ int lens[kMaxBlocks];
-  __shared__ uint32_t keys[kMaxBlocks];
-  __shared__ int totals[3];
-  __shared__ int s_best;
-  const int bh = blockIdx.x, t = threadIdx.x, w = t >> 5, lane = t & 31;
-  const int nw = kPlanThreads / 32, nwords = (nB + 31) / 32;
-  if (!((head_bits >> (bh % H)) & 1ull)) {
-    if (t == 0) head_np[bh] = 0;
+__global__ void __launch_bounds__(256) plan_sizes_kernel(const uint32_t* __restrict__ rowbits, int nB, int H,
+                                                         uint64_t head_bits, int* __restrict__ totals) {
+  const int bh = blockIdx.y, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int a = blockIdx.x * 8 + w;
+  if (!((head_bits >> (bh % H)) & 1ull) || a >= nB) return;
+  const int nwords = (nB + 31) >> 5;
+  const uint32_t* rb = rowbits + static_cast<size_t>(bh) * nB * kWords;
+  const uint32_t wa = lane < nwords ? rb[static_cast<size_t>(a) * kWords + lane] : 0u;
+#pragma unroll
+  for (int si = 0; si < 3; ++si) {
+    const int s = stride_of(si);
+    if (!pair_first(a, s)) continue;
+    const int b = pair_partner(a, s, nB);
+    const uint32_t wb = (b >= 0 && lane < nwords) ? rb[static_cast<size_t>(b) * kWords + lane] : 0u;
+    const int u = __reduce_add_sync(0xffffffffu, __popc(wa | wb));
+    if (lane == 0 && u) atomicAdd(&totals[bh * 3 + si], u);
+  }
+}
+
+__device__ __forceinline__ int best_stride(const int* totals, int bh) {
+  int best = 0;
+  for (int si = 1; si < 3; ++si)
+    if (totals[bh * 3 + si] < totals[bh * 3 + best]) best = si;
+  return stride_of(best);
+}
+
+__global__ void __launch_bounds__(256) plan_unions_kernel(const uint32_t* __restrict__ rowbits, int nB, int H,
+                                                          uint64_t head_bits, const int* __restrict__ totals,
+                                                          int32_t* __restrict__ ulist, int* __restrict__ lens) {
+  const int bh = blockIdx.y, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int a = blockIdx.x * 8 + w;
+  if (!((head_bits >> (bh % H)) & 1ull) || a >= nB) return;
+  const int s = best_stride(totals, bh);
+  if (!pair_first(a, s)) {
+    if (lane == 0) lens[static_cast<size_t>(bh) * nB + a] = -1;
     return;
   }
-  if (t < 3) totals[t] = 0;
+  const int b = pair_partner(a, s, nB);
+  const int nwords = (nB + 31) >> 5;
+  const uint32_t* rb = rowbits + static_cast<size_t>(bh) * nB * kWords;
+  const uint32_t wa = lane < nwords ? rb[static_cast<size_t>(a) * kWords + lane] : 0u;
+  const uint32_t wb = (b >= 0 && lane < nwords) ? rb[static_cast<size_t>(b) * kWords + lane] : 0u;
+  uint32_t un = wa | wb;
+  const int cnt = __popc(un);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int pos = incl - cnt;
+  int32_t* out = ulist + (static_cast<size_t>(bh) * nB + a) * nB;
+  while (un) {  // lane q writes the union entries of key blocks 32q .. 32q+31, ascending
+    const int bit = __ffs(un) - 1;
+    un &= un - 1;
+    const uint32_t mbits = ((wa >> bit) & 1u) | (((wb >> bit) & 1u) << 1);
+    out[pos++] = static_cast<int32_t>((32 * lane + bit) | (mbits << 16));
+  }
+  if (lane == 31) lens[static_cast<size_t>(bh) * nB + a] = incl;
+}
+
+constexpr int kOrderThreads = 512;
+
+// Pairs of a head for stride s: first blocks a with (a / s) even.
+__device__ __forceinline__ int pairs_of(int nB, int s) {
+  return (nB / (2 * s)) * s + min(nB % (2 * s), s);
+}
+
+// Per head: pairs ordered by union length, longest first (rank counting over
+// unique keys), written at the head's offset in the global item list (heads
+// in order; the offset is the closed-form pair count of the heads before).
+__global__ void __launch_bounds__(kOrderThreads) plan_order_kernel(const int* __restrict__ lens,
+                                                                   const int* __restrict__ totals, int nB, int BH,
+                                                                   int H, uint64_t head_bits,
+                                                                   int4* __restrict__ items,
+                                                                   int* __restrict__ n_items) {
+  __shared__ uint32_t keys[kMaxBlocks];
+  __shared__ int nkeys;
+  const int bh = blockIdx.x, t = threadIdx.x;
+  if (bh == 0 && t == 0) {
+    int total = 0;
+    for (int h = 0; h < BH; ++h)
+      if ((head_bits >> (h % H)) & 1ull) total += pairs_of(nB, best_stride(totals, h));
+    *n_items = total;
+  }
+  if (!((head_bits >> (bh % H)) & 1ull)) return;
+  int base = 0;
+  for (int h = 0; h < bh; ++h)
+    if ((head_bits >> (h % H)) & 1ull) base += pairs_of(nB, best_stride(totals, h));
+  if (t == 0) nkeys = 0;
   __syncthreads();
-  // Marks the lists of query blocks a and b (b < 0: none) in this warp's bitmaps.
-  auto mark = [&](int a, int b) {
-    for (int q = lane; q < kMaxBlocks / 32; q += 32) {
-      bm[w][0][q] = 0u;
-      bm[w][1][q] = 0u;
-    }
-    __syncwarp();
-    for (int side = 0; side < 2; ++side) {
-      const int qb = side ? b : a;
-      if (qb < 0) continue;
-      int cnt = counts[static_cast<size_t>(bh) * nB + qb];
-      if (cnt > cap || cnt < 0) {
-        if (lane == 0) atomicOr(err, kErrBadIndex);
-        cnt = cnt < 0 ? 0 : cap;
-      }
-      const int32_t* lst = idx + (static_cast<size_t>(bh) * nB + qb) * cap;
-      for (int e = lane; e < cnt; e += 32) {
-        const int j = lst[e];
-        if (j < 0 || j >= nB) {
-          atomicOr(err, kErrBadIndex);
-          continue;
-        }
-        atomicOr(&bm[w][side][j >> 5], 1u << (j & 31));
-      }
-    }
-    __syncwarp();
-  };
-  const int strides[3] = {1, 2, 4};
-  for (int si = 0; si < 3; ++si) {
-    const int s = strides[si];
-    int local = 0;
-    for (int a = w; a < nB; a += nw) {
-      if ((a / s) & 1) continue;
-      mark(a, pair_partner(a, s, nB));
-      int u = 0;
-      for (int q = lane; q < nwords; q += 32) u += __popc(bm[w][0][q] | bm[w][1][q]);
-      local += __reduce_add_sync(0xffffffffu, u);
-      __syncwarp();
-    }
-    if (lane == 0) atomicAdd(&totals[si], local);
+  for (int a = t; a < nB; a += kOrderThreads) {
+    const int len = lens[static_cast<size_t>(bh) * nB + a];
+    if (len >= 0) keys[atomicAdd(&nkeys, 1)] = (static_cast<uint32_t>(0xFFFF - len) << 16) | static_cast<uint32_t>(a);
   }
   __syncthreads();
-  if (t == 0) {
-    int best = 0;
-    for (int si = 1; si < 3; ++si)
-      if (totals[si] < totals[best]) best = si;
-    s_best = strides[best];
-  }
-  __syncthreads();
-  const int s = s_best;
-  for (int a = t; a < kMaxBlocks; a += kPlanThreads) keys[a] = 0xFFFFFFFFu;
-  __syncthreads();
-  for (int a = w; a < nB; a += nw) {
-    if ((a / s) & 1) continue;
-    const int b = pair_partner(a, s, nB);
-    mark(a, b);
-    // compaction: lane q owns bitmap word q (blocks 32q .. 32q+31), ascending
-    int base = 0;
-    int32_t* out = ulist + (static_cast<size_t>(bh) * nB + a) * nB;
-    for (int q0 = 0; q0 < nwords; q0 += 32) {
-      const int q = q0 + lane;
-      const uint32_t wa = q < nwords ? bm[w][0][q] : 0u;
-      const uint32_t wb = q < nwords ? bm[w][1][q] : 0u;
-      uint32_t un = wa | wb;
-      const int cnt = __popc(un);
-      int incl = cnt;
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      int pos = base + incl - cnt;
-      while (un) {
-        const int bit = __ffs(un) - 1;
-        un &= un - 1;
-        const uint32_t mbits = ((wa >> bit) & 1u) | (((wb >> bit) & 1u) << 1);
-        out[pos++] = static_cast<int32_t>((32 * q + bit) | (mbits << 16));
-      }
-      base += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) {
-      lens[a] = base;
-      keys[a] = (static_cast<uint32_t>(0xFFFF - base) << 16) | static_cast<uint32_t>(a);
-    }
-    __syncwarp();
-  }
-  __syncthreads();
-  // bitonic sort of keys ascending (= union length descending, then a ascending)
-  for (int size = 2; size <= kMaxBlocks; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int e = t; e < kMaxBlocks; e += kPlanThreads) {
-        const int p = e ^ stride;
-        if (p > e) {
-          const bool up = (e & size) == 0;
-          const uint32_t x = keys[e], y = keys[p];
-          if ((x > y) == up) {
-            keys[e] = y;
-            keys[p] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  int np = 0;
-  for (int a = 0; a < nB; ++a) np += ((a / s) & 1) ? 0 : 1;
-  for (int r = t; r < np; r += kPlanThreads) {
-    const int a = static_cast<int>(keys[r] & 0xFFFFu);
+  const int n = nkeys;
+  const int s = best_stride(totals, bh);
+  for (int e = t; e < n; e += kOrderThreads) {
+    const uint32_t k = keys[e];
+    int rank = 0;
+    for (int f = 0; f < n; ++f) rank += keys[f] < k;  // keys are unique: ranks form a permutation
+    const int a = static_cast<int>(k & 0xFFFFu);
     const int b = pair_partner(a, s, nB);
     int4 v;
     v.x = bh;
     v.y = a | ((b < 0 ? kNoBlock : b) << 16);
-    v.z = lens[a];
+    v.z = 0xFFFF - static_cast<int>(k >> 16);
     v.w = static_cast<int>((static_cast<size_t>(bh) * nB + a) * nB);
-    head_items[static_cast<size_t>(bh) * nB + r] = v;
+    items[base + rank] = v;
   }
-  if (t == 0) head_np[bh] = np;
-}
-
-// Concatenates the per-head item lists in head order (one CTA).
-__global__ void __launch_bounds__(1024) compact_items_kernel(const int4* __restrict__ head_items,
-                                                             const int* __restrict__ head_np, int BH, int nB,
-                                                             int4* __restrict__ items, int* __restrict__ n_items) {
-  __shared__ int base_s;
-  if (threadIdx.x == 0) base_s = 0;
-  __syncthreads();
-  for (int bh = 0; bh < BH; ++bh) {
-    const int np = head_np[bh];
-    const int base = base_s;
-    for (int r = threadIdx.x; r < np; r += blockDim.x) items[base + r] = head_items[static_cast<size_t>(bh) * nB + r];
-    __syncthreads();
-    if (threadIdx.x == 0) base_s = base + np;
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) *n_items = base_s;
 }
 
 // Zero output for skipped heads.
@@ -677,6 +802,23 @@ __global__ void zero_heads_kernel(__nv_bfloat16* __restrict__ O, int BH, int H, 
   for (size_t e = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; e < per_head_vec;
        e += static_cast<size_t>(gridDim.x) * blockDim.x)
     dst[e] = z;
+}
+
+// Diagnostic: the polynomial exp2 used for one in four softmax exponentials.
+__global__ void exp2_poly_kernel(const float* __restrict__ y, float* __restrict__ out, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    exp2_poly2(y[i], y[i + 1], out[i], out[i + 1]);
+  } else if (i < n) {
+    float dummy;
+    exp2_poly2(y[i], 0.f, out[i], dummy);
+  }
+}
+
+cudaError_t launch_exp2_poly(const float* y, float* out, int n, cudaStream_t s) {
+  const int pairs = (n + 1) / 2;
+  exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(y, out, n);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- host side
@@ -733,34 +875,41 @@ static cudaError_t launch_attn(const void* Q, const void* K, const void* V, int 
   return launch_attn_kernel<64>(Q, K, V, BH, N, args, s);
 }
 
-cudaError_t launch_sparse_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
-                                    const int32_t* idx, const int32_t* counts, int cap, uint64_t head_bits,
-                                    float scale, void* O, void* ws, cudaStream_t s) {
+cudaError_t launch_attention_plan(const int32_t* idx, const int32_t* counts, int B, int H, int N, int d, int cap,
+                                  uint64_t head_bits, void* ws, cudaStream_t s) {
   const int BH = B * H, nB = N / kBlock;
   const WsLayout wl = ws_layout(B, H, N, d);
   char* base = static_cast<char*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(base + wl.header);
-  int4* head_items = reinterpret_cast<int4*>(base + wl.head_items);
   int4* items = reinterpret_cast<int4*>(base + wl.items);
-  int* head_np = reinterpret_cast<int*>(base + wl.head_np);
   int32_t* ulist = reinterpret_cast<int32_t*>(base + wl.ulist);
-  plan_kernel<<<BH, kPlanThreads, 0, s>>>(idx, counts, nB, cap, H, head_bits, head_items, head_np, ulist,
-                                          &hdr->err);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  compact_items_kernel<<<1, 1024, 0, s>>>(head_items, head_np, BH, nB, items, &hdr->n_items);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  uint32_t* rowbits = reinterpret_cast<uint32_t*>(base + wl.rowbits);
+  int* lens = reinterpret_cast<int*>(base + wl.lens);
+  int* totals = reinterpret_cast<int*>(base + wl.totals);
+  const dim3 grid((nB + 7) / 8, BH);
+  plan_rowbits_kernel<<<grid, 256, 0, s>>>(idx, counts, nB, cap, H, head_bits, rowbits, totals, &hdr->err);
+  plan_sizes_kernel<<<grid, 256, 0, s>>>(rowbits, nB, H, head_bits, totals);
+  plan_unions_kernel<<<grid, 256, 0, s>>>(rowbits, nB, H, head_bits, totals, ulist, lens);
+  plan_order_kernel<<<BH, kOrderThreads, 0, s>>>(lens, totals, nB, BH, H, head_bits, items, &hdr->n_items);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                 uint64_t head_bits, float scale, void* O, void* ws, cudaStream_t s) {
+  const int BH = B * H, nB = N / kBlock;
+  const WsLayout wl = ws_layout(B, H, N, d);
+  char* base = static_cast<char*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(base + wl.header);
   const uint64_t all = (H >= 64) ? ~0ull : ((1ull << H) - 1ull);
   if ((head_bits & all) != all) {
     const size_t per_head_vec = static_cast<size_t>(N) * d / 8;
     zero_heads_kernel<<<dim3(64, BH), 256, 0, s>>>(static_cast<__nv_bfloat16*>(O), BH, H, head_bits, per_head_vec);
-    e = cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   AttnArgs args{};
-  args.items = items;
-  args.ulist = ulist;
+  args.items = reinterpret_cast<const int4*>(base + wl.items);
+  args.ulist = reinterpret_cast<const int32_t*>(base + wl.ulist);
   args.n_items_dev = &hdr->n_items;
   args.n_items_host = 0;
   args.dense = 0;

@@ -79,10 +79,14 @@ constexpr uint64_t kWaitLimitNs = 2000ull * 1000ull * 1000ull;  // 2 s
 // Bounded wait for the phase with the given parity.  On timeout (or when
 // another warp of the CTA has already given up) records kErrTimeout, raises
 // the CTA's abort flag and returns false; the caller unwinds.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err) {
+// sleep_ns > 0 backs off between polls, so a waiting producer or MMA warp
+// does not take issue slots from the softmax warps sharing its SM sub-partition.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
+                                          uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;

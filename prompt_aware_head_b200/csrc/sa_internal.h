@@ -26,9 +26,10 @@ struct WsLayout {
   size_t header = 0;        // WsHeader (256 B)
   size_t qbar = 0, kbar = 0;  // fp32 [BH][nB][d] block means
   size_t items = 0;         // int4 [BH*nB] attention work items (execution order)
-  size_t head_items = 0;    // int4 [BH][nB] per-head items before compaction
-  size_t head_np = 0;       // int32 [BH] items per head
   size_t ulist = 0;         // int32 [BH][nB][nB] union lists (j | bits << 16)
+  size_t rowbits = 0;       // uint32 [BH][nB][32] per-row block bitmaps
+  size_t lens = 0;          // int32 [BH][nB] union length per first block of a pair (-1: not a first)
+  size_t totals = 0;        // int32 [BH][3] summed union length per pairing stride
   size_t total = 0;
 };
 WsLayout ws_layout(int B, int H, int N, int d);
@@ -49,10 +50,13 @@ cudaError_t launch_density(const int32_t* counts, int B, int H, int nB, uint64_t
                            unsigned long long* host_tiles, cudaStream_t s);
 
 // Attention launchers (attention.cu).
-cudaError_t launch_sparse_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
-                                    const int32_t* idx, const int32_t* counts, int cap, uint64_t head_bits,
-                                    float scale, void* O, void* ws, cudaStream_t s);
+cudaError_t launch_attention_plan(const int32_t* idx, const int32_t* counts, int B, int H, int N, int d, int cap,
+                                  uint64_t head_bits, void* ws, cudaStream_t s);
+cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                                 uint64_t head_bits, float scale, void* O, void* ws, cudaStream_t s);
 cudaError_t launch_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
                                    float scale, void* O, void* ws, cudaStream_t s);
+
+cudaError_t launch_exp2_poly(const float* y, float* out, int n, cudaStream_t s);
 
 }  // namespace sa

@@ -307,3 +307,20 @@ def test_density_readback(sa):
     assert da == pytest.approx(ra) and dall == pytest.approx(rall)
     assert st.tiles == 19969 * (w.H - 4) and st.heads_active == w.H - 4
     assert da == pytest.approx(19969 / 264 ** 2)
+
+
+def test_polynomial_exp2_against_cuda(sa):
+    # the softmax's software exponential vs CUDA's exp2 (fp32), relative error bound 1e-4
+    y = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20, device="cuda"),
+                   torch.rand(1 << 20, device="cuda") * 16 - 12]).contiguous()
+    out = torch.empty_like(y)
+    sa.sa_debug_exp2(y, out, y.numel())
+    torch.cuda.synchronize()
+    ref = torch.exp2(y.double())
+    rel = ((out.double() - ref) / ref).abs().max().item()
+    assert rel < 1e-4, rel
+    low = torch.tensor([-200.0, -126.0, -1e30], device="cuda")
+    o2 = torch.empty_like(low)
+    sa.sa_debug_exp2(low, o2, 3)
+    torch.cuda.synchronize()
+    assert torch.all(torch.isfinite(o2)) and torch.all(o2 <= 2.0 ** -124)
