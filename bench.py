@@ -22,7 +22,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -56,94 +55,112 @@ def describe(w, rho):
 
 
 # ------------------------------------------------------------------ oracle (CPU) sample
-def oracle_sample(w, rho, target_s=8.0, seed=0):
-    """Times the fp64 oracle on one head: its full selection plus attention for
-    an evenly spaced subset of its query rows sized for about target_s."""
+def oracle_sample(w, rho, target_s=10.0, seed=0):
+    """Times the fp64 oracle on whole heads of the workload (selection for the
+    head, then attention for all its query rows) until about target_s of CPU
+    work; very long heads are cut to an evenly spaced subset of rows."""
     import oracle
     mask = head_mask_for_layer(w)
-    h = int(np.flatnonzero(mask)[0])
-    Q, K, V = make_qkv(w, seed=seed, heads=[h])
-    Q, K, V = Q[:1], K[:1], V[:1]
-    t0 = time.perf_counter()
+    heads = [int(h) for h in np.flatnonzero(mask)]
     cls = oracle.layout(list(w.segments), w.N)
-    sc = oracle.scores(oracle.pool(Q), oracle.pool(K)).reshape(-1, w.nB, w.nB)
-    idx, cnt = oracle.select(sc, cls, 1, rho)
-    t_sel = time.perf_counter() - t0
-
-    def run(nrows):
-        rows = np.unique(np.linspace(0, w.N - 1, nrows).astype(np.int64))
+    flops = 0.0
+    t_total = 0.0
+    done_heads, done_rows = 0, 0
+    for h in heads:
+        Q, K, V = make_qkv(w, seed=seed, heads=[h])
+        Q, K, V = Q[:1], K[:1], V[:1]
+        t0 = time.perf_counter()
+        sc = oracle.scores(oracle.pool(Q), oracle.pool(K)).reshape(-1, w.nB, w.nB)
+        idx, cnt = oracle.select(sc, cls, 1, rho)
+        t_sel = time.perf_counter() - t0
+        left = max(target_s - t_total - t_sel, 0.5)
+        rows = np.arange(w.N, dtype=np.int64)
+        if done_heads == 0:  # calibrate on the first head
+            t = time.perf_counter()
+            probe = rows[:: max(1, w.N // 512)]
+            oracle.attention(Q, K, V, 1, idx, cnt, rows=probe)
+            per_row = (time.perf_counter() - t) / len(probe)
+            if per_row * w.N > left:
+                rows = np.unique(np.linspace(0, w.N - 1, max(256, int(left / per_row))).astype(np.int64))
         t = time.perf_counter()
         oracle.attention(Q, K, V, 1, idx, cnt, rows=rows)
-        return rows, time.perf_counter() - t
-
-    rows, t = run(256)
-    n = int(min(w.N, max(256, 256 * max(target_s - t_sel, 1.0) / max(t, 1e-6))))
-    rows, t_att = run(n)
-    flops = float(np.sum(4.0 * w.d * 64 * cnt[0, rows // 64]))
-    t_total = t_att + t_sel * len(rows) / w.N
+        t_att = time.perf_counter() - t
+        flops += float(np.sum(4.0 * w.d * 64 * cnt[0, rows // 64]))
+        t_total += t_att + t_sel * len(rows) / w.N
+        done_heads += 1
+        done_rows += len(rows)
+        if t_total >= target_s:
+            break
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     return {
         "value": flops / t_total / 1e12,
         "unit": UNIT,
         "cores": cores,
         "kind": "oracle",
-        "sample": "head %d of the workload: full fp64 selection for the head (%.2f s, charged pro rata) + fp64 "
-                  "attention for %d evenly spaced query rows (%.2f s)" % (h, t_sel, len(rows), t_att),
+        "sample": "%d of %d heads of the workload: fp64 selection per head (charged pro rata to the rows run) + "
+                  "fp64 attention for %d query rows in all (%.1f s)" % (done_heads, len(heads), done_rows, t_total),
         "seconds": t_total,
     }
 
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """Polls SM clock and clock-event reasons through NVML from a thread while
+    the timed region runs (every 2 ms, so short regions still get samples)."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
     def __init__(self, uuid):
         self.uuid = uuid
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_%d.csv" % os.getpid())
+        self.samples = []
+        self.thread = None
+        self.handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            if uuid:
+                u = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+                self.handle = pynvml.nvmlDeviceGetHandleByUUID(u)
+            else:
+                self.handle = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.handle = None
+
+    def _run(self):
+        import threading
+        nv = self.nvml
+        while not self.stop_event.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+                self.samples.append((sm, r))
+            except Exception:
+                pass
+            self.stop_event.wait(0.002)
 
     def start(self):
-        try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                                          "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        if self.handle is None:
+            return
+        import threading
+        self.stop_event = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 8 or (self.uuid and self.uuid not in parts[0]):
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx = max(mx, float(parts[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[4:8]):
-                    if v.lower() == "active":
-                        reasons.add(n)
-        try:
-            os.remove(self.path)
-        except OSError:
-            pass
-        if not sm:
+        self.stop_event.set()
+        self.thread.join(timeout=2)
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        reasons = sorted(n for n, bit in self.REASONS.items() if any(r & bit for _, r in self.samples))
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": float(self.max_mhz),
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml, 2 ms polling"}
 
 
 # ------------------------------------------------------------------ traffic from the committed ncu summary
@@ -390,7 +407,7 @@ def run_reference(args):
     rho = args.density if args.density else w.densities[0]
     per_step = max(2.0, 120.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        oracle_sample(w, rho, target_s=min(per_step, 3.0))
+        oracle_sample(w, rho, target_s=min(per_step, 2.0))
     vals, secs, last = [], [], None
     for _ in range(args.steps):
         last = oracle_sample(w, rho, target_s=per_step)
