@@ -161,6 +161,28 @@ SA_API sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void*
                            void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /*
+ * sa_select_blocks_noalloc: the same selection as sa_select_blocks, for
+ * callers that cannot allocate device memory.  The pages have no counterpart:
+ * this entry point exists for hosts that own all device memory and give
+ * plugins no allocator, and for latency-critical code that must not call
+ * cudaMalloc (which can synchronise the whole device).  It takes no
+ * workspace: the pooled block means live in one fixed array of 16 MiB of
+ * device memory inside the library, which every GPU that loads the library
+ * holds until the process exits.  2 * B * H * nB * d * 4 bytes must fit in
+ * it (e.g. B1 H24 N33280 d128 needs 12.8 MB); larger calls return
+ * SA_ERR_WORKSPACE before anything is launched.  The call allocates nothing.
+ * The first call on a device looks up the array's device address for that
+ * device, so make that first call before any stream capture.  All calls
+ * share the one array, which keeps the last call's contents (each call
+ * overwrites what it reads); calls that overlap on the GPU (two streams, or
+ * two host threads) race on it, so serialise them.  Arguments, outputs and
+ * errors are otherwise those of sa_select_blocks.
+ */
+SA_API sa_status sa_select_blocks_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int d,
+                                          float density, const uint8_t* head_mask, int min_active,
+                                          int32_t* idx, int32_t* counts, float* scores_out, sa_stream_t stream);
+
+/*
  * sa_pattern_mask [SDN "radial control"; GLO sliding window / dilated /
  * global].  Writes the same (idx, counts) a selection would, from a fixed
  * pattern honouring the same pins and drops:

@@ -62,6 +62,7 @@ _SIGS = {
     "sa_layout_release": ([_P], _I),
     "sa_budget": ([_F, _I], _I),
     "sa_select_blocks": ([_P, _P, _P, _I, _I, _I, _F, _P, _I, _P, _P, _P, _P, _SZ, _P], _I),
+    "sa_select_blocks_noalloc": ([_P, _P, _P, _I, _I, _I, _F, _P, _I, _P, _P, _P, _P], _I),
     "sa_pattern_mask": ([_P, ctypes.POINTER(sa_pattern), _I, _I, _F, _P, _I, _P, _P, _P], _I),
     "sa_block_sparse_attention": ([_P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _F, _P, _P, _SZ, _P], _I),
     "sa_attention_plan": ([_P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _SZ, _P], _I),
@@ -180,6 +181,16 @@ def sa_select_blocks(L: Layout, Q, K, B: int, H: int, d: int, density: float, he
     _check(_lib.sa_select_blocks(L.handle, _addr(Q), _addr(K), B, H, d, ctypes.c_float(density), mptr, min_active,
                                  _addr(idx), _addr(counts), _addr(scores_out), _addr(ws), ws_bytes, _stream(stream)),
            "sa_select_blocks")
+
+
+def sa_select_blocks_noalloc(L: Layout, Q, K, B: int, H: int, d: int, density: float, head_mask, min_active: int,
+                             idx, counts, scores_out, stream=None) -> None:
+    """sa_select_blocks without a workspace, for callers that cannot allocate
+    device memory (its scratch is a fixed 16 MiB array inside the library)."""
+    mptr, _keep = _host_mask(head_mask)
+    _check(_lib.sa_select_blocks_noalloc(L.handle, _addr(Q), _addr(K), B, H, d, ctypes.c_float(density), mptr,
+                                         min_active, _addr(idx), _addr(counts), _addr(scores_out), _stream(stream)),
+           "sa_select_blocks_noalloc")
 
 
 def sa_pattern_mask(L: Layout, kind: int, B: int, H: int, density: float = 1.0, head_mask=None,

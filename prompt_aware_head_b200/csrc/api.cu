@@ -282,6 +282,28 @@ sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void* K, int
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+sa_status sa_select_blocks_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int d,
+                                   float density, const uint8_t* head_mask, int min_active, int32_t* idx,
+                                   int32_t* counts, float* scores_out, sa_stream_t stream) {
+  if (!L || !Q || !K || !idx || !counts) return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K)) return SA_ERR_INVALID_ARG;
+  if (B <= 0 || (d != 64 && d != 128)) return SA_ERR_SHAPE;
+  if (static_cast<long long>(B) * H * L->N >= (1ll << 31)) return SA_ERR_SHAPE;
+  if (!density_ok(density)) return SA_ERR_INVALID_ARG;
+  uint64_t bits = 0;
+  sa_status st = head_bits_of(head_mask, H, min_active, &bits);
+  if (st != SA_OK) return st;
+  // the pooled block means (q-bar and k-bar, fp32) must fit the fixed scratch
+  const size_t need = 2ull * B * H * L->nB * d * sizeof(float);
+  if (need > select_noalloc_limit()) return SA_ERR_WORKSPACE;
+  DeviceInfo di;
+  if ((st = check_device(&di)) != SA_OK) return st;
+  if (di.id != L->device) return SA_ERR_INVALID_ARG;
+  const int k = sa_budget(density, L->n_cand);
+  return from_cuda(launch_select_noalloc(L, Q, K, B, H, d, k, bits, idx, counts, scores_out,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H, float density,
                           const uint8_t* head_mask, int min_active, int32_t* idx, int32_t* counts,
                           sa_stream_t stream) {

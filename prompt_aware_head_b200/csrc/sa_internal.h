@@ -43,6 +43,11 @@ cudaError_t device_info(DeviceInfo* out);
 cudaError_t launch_select(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, int k,
                           uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out, void* ws,
                           cudaStream_t s);
+// Selection with its scratch in a fixed device array (no workspace).
+size_t select_noalloc_limit();
+cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, int k,
+                                  uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out,
+                                  cudaStream_t s);
 // kind: 0 radial, 1 window+global, 2 dilated, 3 dense (every non-drop block).
 cudaError_t launch_pattern(const sa_layout* L, int kind, int W, int G, int r, int k, int B, int H,
                            uint64_t head_bits, int32_t* idx, int32_t* counts, cudaStream_t s);

@@ -393,6 +393,65 @@ cudaError_t launch_select(const sa_layout* L, const void* Q, const void* K, int 
   return launch_score_select_d<64>(nc, qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
 }
 
+// ============================================================== selection without allocation
+// For callers that cannot allocate device memory (see sa_select_blocks_noalloc
+// in sa.h): the pooled block means live in this fixed, file-scope device
+// array instead of the caller's workspace.  Every process that loads the
+// library holds it on every GPU it uses until exit.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB: q-bar and k-bar, fp32
+static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
+
+size_t select_noalloc_limit() { return kNoAllocScratchBytes; }
+
+// Device address of the scratch array for the current device.  The host-side
+// symbol is only a stand-in, so the address is asked of the runtime once per
+// device (on the first call made with that device current) and cached.
+static cudaError_t noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_select_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, int k,
+                                  uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out,
+                                  cudaStream_t s) {
+  const int BH = B * H, nB = L->nB;
+  const int nc = chunks_for(nB);
+  if (nc < 0) return cudaErrorInvalidValue;
+  if (k >= L->n_cand && scores_out == nullptr)  // dense lists: no scratch used
+    return launch_pattern(L, 3, 0, 0, 1, k, B, H, head_bits, idx, counts, s);
+  void* scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  // q-bar and k-bar are written in full for every active head by the pooling
+  // kernel before the scoring kernel reads them: nothing needs clearing.
+  float* qbar = static_cast<float*>(scratch);
+  float* kbar = qbar + static_cast<size_t>(BH) * nB * d;
+  dim3 pgrid(nB, BH);
+  if (d == 128)
+    pool_kernel<128><<<pgrid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
+                                           qbar, kbar, L->N, nB, H, head_bits);
+  else
+    pool_kernel<64><<<pgrid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
+                                          qbar, kbar, L->N, nB, H, head_bits);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (d == 128) return launch_score_select_d<128>(nc, qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
+  return launch_score_select_d<64>(nc, qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
+}
+
 template <int NC>
 static void launch_pattern_t(const sa_layout* L, int kind, int W, int G, int r, int k, int BH, int H,
                              uint64_t head_bits, int32_t* idx, int32_t* counts, cudaStream_t s) {
