@@ -259,6 +259,7 @@ sa_status sa_check(void* ws, sa_stream_t stream) {
   if (err && cudaMemset(&static_cast<WsHeader*>(ws)->err, 0, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
   if (err & kErrBadIndex) return SA_ERR_BAD_INDEX;
   if (err & kErrTimeout) return SA_ERR_TIMEOUT;
+  if (err & kErrSmemAlign) return SA_ERR_UNSUPPORTED;
   return SA_OK;
 }
 

@@ -51,7 +51,7 @@ struct AttnArgs {
   int* err;
 };
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA issuer, 8 softmax warps
 constexpr int kNoBlock = 0xFFFF;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t kBackoffNs = 40;            // producer / MMA poll back-off  // log2 units: rescale O when the max grows by > 2^8
@@ -131,28 +131,33 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t adesc, uint64
   }
 }
 
-// O += P V for one step of 64 * nblk keys: A = P (bf16 in TMEM, 8 columns
-// per 16 keys), B = V pair (MN-major SW128 smem; 16 keys = 2 KB per slice).
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate, int nblk) {
+// O_c += P_c V_c for the step's key blocks c = 0 (and 1 when nblk = 2): each
+// key block accumulates into its own O (TMEM columns d0 / d1), so the two
+// softmax warps that own a row's two blocks keep independent running maxima.
+// A = P (bf16 in TMEM, 8 columns per 16 keys; each block's P sits in the
+// first half of that block's own 64 S columns, so block 1's starts 64 in),
+// B = V pair (MN-major SW128 smem; 16 keys = 2 KB per slice, block 1 starts
+// 8 KB in).
+__device__ __forceinline__ void issue_pv(uint32_t d0, uint32_t d1, uint32_t a_tmem, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate, int nblk) {
   if (nblk == 2) {
     asm volatile(
         "{\n .reg .pred p0, p1;\n .reg .b32 t1, t2, t3, t4, t5, t6, t7;\n"
         " .reg .b64 b1, b2, b3, b4, b5, b6, b7;\n"
-        " setp.ne.b32 p0, %4, 0;\n setp.eq.b32 p1, 0, 0;\n"
-        " add.u32 t1, %1, 8;\n add.u32 t2, %1, 16;\n add.u32 t3, %1, 24;\n add.u32 t4, %1, 32;\n"
-        " add.u32 t5, %1, 40;\n add.u32 t6, %1, 48;\n add.u32 t7, %1, 56;\n"
-        " add.s64 b1, %2, 128;\n add.s64 b2, %2, 256;\n add.s64 b3, %2, 384;\n add.s64 b4, %2, 512;\n"
-        " add.s64 b5, %2, 640;\n add.s64 b6, %2, 768;\n add.s64 b7, %2, 896;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t1], b1, %3, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t2], b2, %3, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t3], b3, %3, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t4], b4, %3, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t5], b5, %3, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t6], b6, %3, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t7], b7, %3, p1;\n}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        " setp.ne.b32 p0, %5, 0;\n setp.eq.b32 p1, 0, 0;\n"
+        " add.u32 t1, %2, 8;\n add.u32 t2, %2, 16;\n add.u32 t3, %2, 24;\n add.u32 t4, %2, 64;\n"
+        " add.u32 t5, %2, 72;\n add.u32 t6, %2, 80;\n add.u32 t7, %2, 88;\n"
+        " add.s64 b1, %3, 128;\n add.s64 b2, %3, 256;\n add.s64 b3, %3, 384;\n add.s64 b4, %3, 512;\n"
+        " add.s64 b5, %3, 640;\n add.s64 b6, %3, 768;\n add.s64 b7, %3, 896;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %3, %4, p0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t1], b1, %4, p1;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t2], b2, %4, p1;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t3], b3, %4, p1;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t4], b4, %4, p0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t5], b5, %4, p1;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t6], b6, %4, p1;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t7], b7, %4, p1;\n}\n" ::"r"(d0),
+        "r"(d1), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
   } else {
     asm volatile(
@@ -163,7 +168,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint6
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p0;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [t1], b1, %3, p1;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [t2], b2, %3, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t3], b3, %3, p1;\n}\n" ::"r"(d_tmem),
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t3], b3, %3, p1;\n}\n" ::"r"(d0),
         "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
   }
@@ -276,10 +281,14 @@ struct AttnSmem {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kQBuf * kTile;
   static constexpr int kV = kK + kNK * kTile;
-  static constexpr int kBar = kV + kNV * kTile;
-  static constexpr int kBytes = kBar + 512;      // barriers + flags
-  static constexpr int kAlloc = kBytes + 1024;   // slack for 1024-B alignment
-  static_assert(kAlloc <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
+  static constexpr int kBar = kV + kNV * kTile;     // mbarriers + flags (512 B)
+  static constexpr int kX = kBar + 512;              // softmax pair exchange: [2][4][2][32] floats
+  static constexpr int kBytes = kX + 2048;
+  // The dynamic shared memory window starts 1 KB-aligned when a kernel has no
+  // static shared memory; the slack covers a smaller alignment, and the kernel
+  // checks the padding it needs against it before touching anything.
+  static constexpr int kAlloc = (kBytes + 1024 <= 232448) ? kBytes + 1024 : 232448;
+  static_assert(kBytes <= kAlloc, "dynamic shared memory above the 227 KB per-CTA limit");
 };
 
 template <int D>
@@ -289,8 +298,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   using S = AttnSmem<D>;
   constexpr int NK = S::kNK, NV = S::kNV, QB = S::kQBuf;
   constexpr uint32_t kTxBlock = 64 * D * 2;  // bytes of one 64-row block
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  if (pad + S::kBytes > static_cast<uint32_t>(S::kAlloc)) {  // uniform across the CTA: nothing started yet
+    if (threadIdx.x == 0) atomicOr(a.err, kErrSmemAlign);
+    return;
+  }
+  uint8_t* sm = smem_raw + pad;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + S::kBar);
   uint64_t* q_full = bars + 0;              // [QB]
   uint64_t* q_empty = bars + 2;             // [QB] after the last S MMA of an item
@@ -303,7 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_empty = k_full + NK;          // [NK] after the S MMA that read the stage
   uint64_t* v_full = k_empty + NK;          // [NV]
   uint64_t* v_empty = v_full + NV;          // [NV] after the PV MMA that read the stage
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(v_empty + NV);
+  uint64_t* pair_x = v_empty + NV;          // [2 step parities][4 quads]: block-max exchange
+  uint64_t* pair_l = pair_x + 8;            // [4 quads]: row-sum exchange at the end of an item
+  uint64_t* pair_g = pair_l + 4;            // [4 quads]: exchange slot released
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pair_g + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -312,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], 8);
     }
     mbar_init(o_done, 1);
     mbar_init(o_final, 1);
@@ -324,6 +341,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < NV; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 8; ++i) mbar_init(&pair_x[i], 2);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&pair_l[i], 2);
+      mbar_init(&pair_g[i], 2);
     }
     *abort_flag = 0;
     mbar_fence_init();
@@ -419,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&v_full[vst], (pg / NV) & 1, abort_flag, a.err, kBackoffNs)) return false;
         tc_fence_after();
         const uint64_t bdesc = smem_desc_sw128(smem_u32(sm + S::kV + vst * S::kTile), S::kChunk, 1024);
-        issue_pv(tm + 256, tm + (pg & 1) * 128, bdesc, idesc_pv, pacc, pnblk);
+        issue_pv(tm + 256, tm + 384, tm + (pg & 1) * 128, bdesc, idesc_pv, pacc, pnblk);
         tc_commit(&v_empty[vst]);
         tc_commit(o_done);
         if (plast) tc_commit(o_final);
@@ -461,11 +483,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ======================= softmax / epilogue (warps 2..5) =======================
+    // ======================= softmax / epilogue (warps 2..9) =======================
+    // Two warps per TMEM lane quadrant: warp (quad, cb) owns the 32 tile rows
+    // of its quadrant and key block cb of every step (S columns 64*cb ..,
+    // P columns 64*cb .. 64*cb+31, accumulator O_cb at TMEM column 256 + 128*cb).  Each
+    // runs its own online softmax (running max m, sum l) with no per-step
+    // synchronisation; the two partial results of a row are merged once per
+    // item in the epilogue:  O = (w0 O_0 + w1 O_1) / (w0 l_0 + w1 l_1),
+    // w_c = 2^(m_c - max(m_0, m_1)).
+    const int sw = warp - 2;                   // 0..7
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+    const int cb = sw >> 2;                    // key block of the step this warp handles
     const int row = quad * 32 + lane;          // tile row = TMEM lane
     const int half = row >> 6;                 // 0: query block i0, 1: i1
     const uint32_t t_lane = tm + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t o_own = t_lane + 256 + 128 * cb;
+    constexpr int DH = D / 2;                  // output columns this warp writes
+    float* xbuf = reinterpret_cast<float*>(sm + S::kX);  // [4 quads][2 warps][2 values][32 lanes]
     const float c = a.scale_log2;
     uint32_t g = 0, t = 0;
     bool ok = true;
@@ -476,147 +510,129 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nsteps = (it.len + 1) >> 1;
       const int qblk = half ? it.i1 : it.i0;
       const bool row_valid = qblk != kNoBlock;
-      __nv_bfloat16* orow = a.O + (static_cast<size_t>(it.bh) * a.N + static_cast<size_t>(qblk) * 64 + (row & 63)) * D;
+      __nv_bfloat16* orow =
+          a.O + (static_cast<size_t>(it.bh) * a.N + static_cast<size_t>(qblk) * 64 + (row & 63)) * D + cb * DH;
       if (nsteps == 0) {
         if (row_valid) {
-          uint4 z = make_uint4(0, 0, 0, 0);
+          const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int q = 0; q < D / 8; ++q) reinterpret_cast<uint4*>(orow)[q] = z;
+          for (int q = 0; q < DH / 8; ++q) reinterpret_cast<uint4*>(orow)[q] = z;
         }
         continue;
       }
       float m = -INFINITY, l = 0.f;
-      // union entries are prefetched one step ahead (global loads off the critical path)
-      uint32_t e0n = load_entry(a, it, 0);
-      uint32_t e1n = it.len > 1 ? load_entry(a, it, 1) : 0u;
+      // this warp's union entry per step, prefetched one step ahead
+      uint32_t en = cb < it.len ? load_entry(a, it, cb) : 0u;
       for (int s = 0; s < nsteps; ++s, ++g) {
         const int sb = g & 1;
         const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
-        const uint32_t e0 = e0n, e1 = nblk == 2 ? e1n : 0u;
-        if (2 * s + 2 < it.len) e0n = load_entry(a, it, 2 * s + 2);
-        if (2 * s + 3 < it.len) e1n = load_entry(a, it, 2 * s + 3);
+        const bool present = cb < nblk;        // this warp's key block exists in the step
+        const uint32_t e = present ? en : 0u;
+        if (2 * s + 2 + cb < it.len) en = load_entry(a, it, 2 * s + 2 + cb);
         if (!warp_wait(&s_full[sb], (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
         tc_fence_after();
-        const bool b0 = (e0 >> (16 + half)) & 1u;
-        const bool b1 = (e1 >> (16 + half)) & 1u;
-        const uint32_t s_col = t_lane + sb * 128;
-        uint32_t x[128];
-        uint32_t pk[64];
-        float sv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        float mv0 = -INFINITY, mv1 = -INFINITY;
-        float sum = 0.f, alpha = 1.f;
+        const bool bm = (e >> (16 + half)) & 1u;  // this half's query block selected the key block
+        uint32_t pk[32];
+        float alpha = 1.f, sum = 0.f;
         bool rescale = false;
-        if (!(b0 || b1)) {
-#pragma unroll
-          for (int q = 0; q < 64; ++q) pk[q] = 0u;
-        } else if (__any_sync(0xffffffffu, m == -INFINITY)) {
-          // first selected block of this half (warp-uniform): find the max first
-          if (b0) {
-            tmem_ld32(s_col, x);
-            tmem_ld32(s_col + 32, x + 32);
-          }
-          if (b1) {
-            tmem_ld32(s_col + 64, x + 64);
-            tmem_ld32(s_col + 96, x + 96);
-          }
+        if (bm) {
+          uint32_t x[64];
+          const uint32_t s_col = t_lane + sb * 128 + cb * 64;
+          tmem_ld32(s_col, x);
+          tmem_ld32(s_col + 32, x + 32);
           tmem_wait_ld();
-          const float m_new = fmaxf(m, row_max(x, b0, b1) * c);  // c > 0: max commutes with the scaling
-          rescale = m != -INFINITY && m_new > m;
-          alpha = rescale ? ex2(m - m_new) : 1.f;
-          m = m_new;
-          if (b0) exp_half<false>(x, c, m, pk, sv, mv0, mv1);
-          else {
+          float mv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int q = 0; q < 32; ++q) pk[q] = 0u;
+          for (int q = 0; q < 32; ++q)
+            mv[q & 3] = max3f(mv[q & 3], __uint_as_float(x[2 * q]), __uint_as_float(x[2 * q + 1]));
+          const float mx = fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])) * c;  // c > 0
+          // Running max: set by the first selected block, raised again only
+          // when it grows by more than 2^8 (then O_cb is rescaled); otherwise
+          // the stale max is kept (exact after the final division by the sum).
+          if (m == -INFINITY) {
+            m = mx;
+          } else if (mx > m + kRescaleThreshold) {
+            alpha = ex2(m - mx);
+            m = mx;
+            rescale = true;
           }
-          if (b1) exp_half<false>(x + 64, c, m, pk + 32, sv, mv0, mv1);
-          else {
-#pragma unroll
-            for (int q = 32; q < 64; ++q) pk[q] = 0u;
-          }
+          float sv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          float mv0 = 0.f, mv1 = 0.f;
+          exp_half<false>(x, c, m, pk, sv, mv0, mv1);
           sum = sum8(sv);
         } else {
-          // Fused pass with the running (possibly stale) max m; the first
-          // half's exponentials overlap the second half's TMEM load.  Only
-          // when a row's max grows by more than 2^8 is the pass redone with
-          // the new max and O rescaled.
-          if (b0) {
-            tmem_ld32(s_col, x);
-            tmem_ld32(s_col + 32, x + 32);
-            tmem_wait_ld();
-          }
-          if (b1) {
-            tmem_ld32(s_col + 64, x + 64);
-            tmem_ld32(s_col + 96, x + 96);
-          }
-          if (b0) exp_half<true>(x, c, m, pk, sv, mv0, mv1);
-          else {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) pk[q] = 0u;
-          }
-          if (b1) {
-            tmem_wait_ld();
-            exp_half<true>(x + 64, c, m, pk + 32, sv, mv0, mv1);
-          } else {
-#pragma unroll
-            for (int q = 32; q < 64; ++q) pk[q] = 0u;
-          }
-          sum = sum8(sv);
-          const float mx = fmaxf(mv0, mv1) * c;
-          rescale = mx > m + kRescaleThreshold;
-          if (__any_sync(0xffffffffu, rescale)) {
-            const float m_new = rescale ? mx : m;
-            alpha = rescale ? ex2(m - m_new) : 1.f;
-            m = m_new;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) sv[u] = 0.f;
-            if (b0) exp_half<false>(x, c, m, pk, sv, mv0, mv1);
-            if (b1) exp_half<false>(x + 64, c, m, pk + 32, sv, mv0, mv1);
-            sum = sum8(sv);
-          }
+          for (int q = 0; q < 32; ++q) pk[q] = 0u;
         }
         l = l * alpha + sum;
         if (__any_sync(0xffffffffu, rescale)) {
-          // O (TMEM) holds PV results up to step g-1: wait for PV_{g-1}, then scale.
+          // O_cb holds PV results up to step g-1: wait for PV_{g-1}, then scale.
           if (!warp_wait(o_done, (g - 1) & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int cc = 0; cc < D; cc += 32) {
             uint32_t o[32];
-            tmem_ld32(t_lane + 256 + cc, o);
+            tmem_ld32(o_own + cc, o);
             tmem_wait_ld();
 #pragma unroll
             for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-            tmem_st32(t_lane + 256 + cc, o);
+            tmem_st32(o_own + cc, o);
           }
         }
-        tmem_st32(s_col, pk);
-        if (nblk == 2) tmem_st32(s_col + 32, pk + 32);
+        // P of this key block (bf16 pairs) over the first half of the block's own
+        // S columns, which only this warp reads: no race with the partner warp.
+        if (present) tmem_st32(t_lane + sb * 128 + cb * 64, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[sb]);
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 -> global
+      // epilogue: merge the two partial results of each row, O -> bf16 -> global
+      float* xm = xbuf + (quad * 2) * 64;        // [2 warps][m, l][32]
+      xm[cb * 64 + lane] = m;
+      xm[cb * 64 + 32 + lane] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pair_l[quad]);
+      if (!warp_wait(&pair_l[quad], t & 1, abort_flag, a.err)) { ok = false; break; }
+      const float m_o = xm[(1 - cb) * 64 + lane], l_o = xm[(1 - cb) * 64 + 32 + lane];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pair_g[quad]);  // both read: the slot may be written again
+      if (!warp_wait(&pair_g[quad], t & 1, abort_flag, a.err)) { ok = false; break; }
+      const float m0 = cb ? m_o : m, l0 = cb ? l_o : l, m1 = cb ? m : m_o, l1 = cb ? l : l_o;
+      const bool o1_valid = it.len >= 2;         // O_1 is only written when a step has two blocks
+      const float mmax = fmaxf(m0, o1_valid ? m1 : -INFINITY);
+      const float w0 = l0 > 0.f ? ex2(m0 - mmax) : 0.f;
+      const float w1 = (o1_valid && l1 > 0.f) ? ex2(m1 - mmax) : 0.f;
+      const float lt = w0 * l0 + w1 * l1;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float f0 = w0 * inv, f1 = w1 * inv;
+      const bool any_w1 = __any_sync(0xffffffffu, w1 != 0.f);
       if (!warp_wait(o_final, t & 1, abort_flag, a.err)) { ok = false; break; }
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-      for (int cc = 0; cc < D; cc += 32) {
-        uint32_t o[32];
-        tmem_ld32(t_lane + 256 + cc, o);
+      for (int cc = 0; cc < DH; cc += 32) {
+        uint32_t o0[32], o1[32];
+        tmem_ld32(t_lane + 256 + cb * DH + cc, o0);
+        if (o1_valid) tmem_ld32(t_lane + 384 + cb * DH + cc, o1);
         tmem_wait_ld();
+        float v[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(o0[q]) * f0;
+        if (any_w1) {  // rows with w1 == 0 never read O_1 (it may be stale when unused)
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[q] = (w1 != 0.f) ? fmaf(__uint_as_float(o1[q]), f1, v[q]) : v[q];
+        }
         if (row_valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + cc);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
-            dst[q] = v;
+            uint4 u;
+            u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+            u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+            u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+            u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+            dst[q] = u;
           }
         }
       }

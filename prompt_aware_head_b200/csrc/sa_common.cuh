@@ -17,7 +17,7 @@ constexpr int kMaxHeads = 64;           // head_mask bits
 enum BlockClass : uint8_t { kPin = 0, kSparse = 1, kDrop = 2 };
 
 // Error bits in the workspace header (mapped to sa_status by the host).
-enum ErrBits : int { kErrBadIndex = 1, kErrTimeout = 2 };
+enum ErrBits : int { kErrBadIndex = 1, kErrTimeout = 2, kErrSmemAlign = 4 };
 
 // Workspace header (first 256 bytes of the caller's workspace).
 struct WsHeader {
