@@ -21,8 +21,9 @@
 //    d/16 SS MMAs into TMEM; P is written back to TMEM as bf16 and
 //    O += P V is one asm block of TS MMAs (A from TMEM).  S is double
 //    buffered in TMEM so the MMAs of step g+1 overlap the softmax of step g.
-//  * Warp roles: warp 0 TMA producer, warp 1 MMA issuer (one thread), warps
-//    2-5 softmax / correction / epilogue (one thread per tile row).
+//  * Warp roles: warp 0 TMA producer for Q and K, warp 10 TMA producer for V,
+//    warp 1 MMA issuer (one thread), warps 2-9 softmax / correction /
+//    epilogue (two warps per tile row, one per key block of a step).
 //  * Rescaling of O (in TMEM) happens only when a row's running max grows by
 //    more than 2^8; otherwise the stale max is kept (exact after the final
 //    division by the running sum).
@@ -51,14 +52,25 @@ struct AttnArgs {
   int* err;
 };
 
-constexpr int kThreads = 320;  // producer, MMA issuer, 8 softmax warps
+constexpr int kThreads = 352;  // Q/K producer, MMA issuer, 8 softmax warps, V producer
 constexpr int kNoBlock = 0xFFFF;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t kBackoffNs = 40;            // producer / MMA poll back-off  // log2 units: rescale O when the max grows by > 2^8
 
 struct Item {
   int bh, i0, i1, len, off;
+  int rot;  // the item walks its union list starting at entry rot (wrapping)
 };
+
+// Online softmax is exact in any key-block order, so each item starts its
+// walk at an item-dependent offset: CTAs working on the same head then read
+// different K/V blocks at any moment instead of all sweeping the same ones
+// (which throttles L2).  The offset is a hash of (head, query block).
+__device__ __forceinline__ int item_rotation(int bh, int i0, int len) {
+  if (len <= 1) return 0;
+  const uint32_t h = (static_cast<uint32_t>(bh) * 0x9E3779B1u) ^ (static_cast<uint32_t>(i0 + 1) * 0x85EBCA77u);
+  return static_cast<int>((h >> 7) % static_cast<uint32_t>(len));
+}
 
 __device__ __forceinline__ Item load_item(const AttnArgs& a, int k) {
   Item it;
@@ -77,14 +89,17 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int k) {
     it.len = v.z;
     it.off = v.w;
   }
+  it.rot = item_rotation(it.bh, it.i0, it.len);
   return it;
 }
 
 // Union entry e of an item: key block j in the low 16 bits, membership bits
 // (bit 16: query block i0 selected j, bit 17: i1 selected j).
 __device__ __forceinline__ uint32_t load_entry(const AttnArgs& a, const Item& it, int e) {
-  if (a.dense) return static_cast<uint32_t>(e) | ((it.i1 == kNoBlock ? 1u : 3u) << 16);
-  return static_cast<uint32_t>(a.ulist[it.off + e]);
+  int pos = e + it.rot;  // e < len, rot < len
+  if (pos >= it.len) pos -= it.len;
+  if (a.dense) return static_cast<uint32_t>(pos) | ((it.i1 == kNoBlock ? 1u : 3u) << 16);
+  return static_cast<uint32_t>(a.ulist[it.off + pos]);
 }
 
 __device__ __forceinline__ int item_index(int r, int cta, int G) {
@@ -136,28 +151,28 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t adesc, uint64
 // softmax warps that own a row's two blocks keep independent running maxima.
 // A = P (bf16 in TMEM, 8 columns per 16 keys; each block's P sits in the
 // first half of that block's own 64 S columns, so block 1's starts 64 in),
-// B = V pair (MN-major SW128 smem; 16 keys = 2 KB per slice, block 1 starts
-// 8 KB in).
-__device__ __forceinline__ void issue_pv(uint32_t d0, uint32_t d1, uint32_t a_tmem, uint64_t bdesc,
+// B = the block's V (MN-major SW128 smem [d/64 chunks][64 keys][128 B];
+// 16 keys = 2 KB per slice; bdesc0 / bdesc1 address blocks 0 / 1).
+__device__ __forceinline__ void issue_pv(uint32_t d0, uint32_t d1, uint32_t a_tmem, uint64_t bdesc0, uint64_t bdesc1,
                                          uint32_t idesc, uint32_t accumulate, int nblk) {
   if (nblk == 2) {
     asm volatile(
         "{\n .reg .pred p0, p1;\n .reg .b32 t1, t2, t3, t4, t5, t6, t7;\n"
-        " .reg .b64 b1, b2, b3, b4, b5, b6, b7;\n"
-        " setp.ne.b32 p0, %5, 0;\n setp.eq.b32 p1, 0, 0;\n"
+        " .reg .b64 b1, b2, b3, b5, b6, b7;\n"
+        " setp.ne.b32 p0, %6, 0;\n setp.eq.b32 p1, 0, 0;\n"
         " add.u32 t1, %2, 8;\n add.u32 t2, %2, 16;\n add.u32 t3, %2, 24;\n add.u32 t4, %2, 64;\n"
         " add.u32 t5, %2, 72;\n add.u32 t6, %2, 80;\n add.u32 t7, %2, 88;\n"
-        " add.s64 b1, %3, 128;\n add.s64 b2, %3, 256;\n add.s64 b3, %3, 384;\n add.s64 b4, %3, 512;\n"
-        " add.s64 b5, %3, 640;\n add.s64 b6, %3, 768;\n add.s64 b7, %3, 896;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %3, %4, p0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t1], b1, %4, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t2], b2, %4, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t3], b3, %4, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t4], b4, %4, p0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t5], b5, %4, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t6], b6, %4, p1;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t7], b7, %4, p1;\n}\n" ::"r"(d0),
-        "r"(d1), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        " add.s64 b1, %3, 128;\n add.s64 b2, %3, 256;\n add.s64 b3, %3, 384;\n"
+        " add.s64 b5, %4, 128;\n add.s64 b6, %4, 256;\n add.s64 b7, %4, 384;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %3, %5, p0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t1], b1, %5, p1;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t2], b2, %5, p1;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [t3], b3, %5, p1;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t4], %4, %5, p0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t5], b5, %5, p1;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t6], b6, %5, p1;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%1], [t7], b7, %5, p1;\n}\n" ::"r"(d0),
+        "r"(d1), "r"(a_tmem), "l"(bdesc0), "l"(bdesc1), "r"(idesc), "r"(accumulate)
         : "memory");
   } else {
     asm volatile(
@@ -169,7 +184,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d0, uint32_t d1, uint32_t a_tm
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [t1], b1, %3, p1;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [t2], b2, %3, p1;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [t3], b3, %3, p1;\n}\n" ::"r"(d0),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        "r"(a_tmem), "l"(bdesc0), "r"(idesc), "r"(accumulate)
         : "memory");
   }
 }
@@ -271,6 +286,7 @@ __device__ __forceinline__ float row_max(const uint32_t (&x)[128], bool b0, bool
 template <int D>
 struct AttnSmem {
   static constexpr int kTile = 128 * D * 2;      // 128 rows x D bf16 (a Q tile, or a K / V pair)
+  static constexpr int kVBlock = 64 * D * 2;     // one V block, laid out [D/64 chunks][64 keys][128 B]
   static constexpr int kChunk = 128 * 128;       // one 64-column chunk of a 128-row tile
   // K and V live in separate rings: a K stage is free as soon as its S MMA
   // completes, a V stage once its PV MMA does.  Three stages each cover the
@@ -310,7 +326,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_empty = bars + 2;             // [QB] after the last S MMA of an item
   uint64_t* s_full = bars + 4;              // [2]
   uint64_t* p_full = bars + 6;              // [2]
-  uint64_t* o_done = bars + 8;              // after every PV
   uint64_t* o_final = bars + 9;             // after the last PV of an item
   uint64_t* drain = bars + 10;              // abort path
   uint64_t* k_full = bars + 12;             // [NK]
@@ -331,7 +346,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 8);
     }
-    mbar_init(o_done, 1);
     mbar_init(o_final, 1);
     mbar_init(drain, 1);
     for (int i = 0; i < NK; ++i) {
@@ -362,12 +376,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total = a.dense ? a.n_items_host : *reinterpret_cast<const volatile int*>(a.n_items_dev);
 
   if (warp == 0) {
-    // ======================= TMA producer =======================
+    // ======================= TMA producer: Q and K =======================
     if (lane == 0) {
       uint32_t g = 0, t = 0;
-      int k_phase[NK], v_phase[NV], q_phase[2] = {-1, -1};
+      int k_phase[NK], q_phase[2] = {-1, -1};
       for (int i = 0; i < NK; ++i) k_phase[i] = -1;
-      for (int i = 0; i < NV; ++i) v_phase[i] = -1;
       bool ok = true;
       for (int r = 0; ok; ++r) {
         const int k = item_index(r, cta, G);
@@ -387,10 +400,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (it.i1 != kNoBlock) tma_load_2d(qdst + c * S::kChunk + 8192, &tmQ, 64 * c, row0 + 64 * it.i1, &q_full[qb]);
         }
         q_phase[qb] = uq & 1;
+        // union entries are prefetched one step ahead: the TMA coordinates of a
+        // step then never wait on a global load
+        uint32_t e0n = load_entry(a, it, 0);
+        uint32_t e1n = it.len > 1 ? load_entry(a, it, 1) : 0u;
         for (int s = 0; s < nsteps; ++s, ++g) {
-          const uint32_t e0 = load_entry(a, it, 2 * s);
           const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
-          const uint32_t e1 = nblk == 2 ? load_entry(a, it, 2 * s + 1) : 0u;
+          const uint32_t e0 = e0n, e1 = nblk == 2 ? e1n : 0u;
+          if (2 * s + 2 < it.len) e0n = load_entry(a, it, 2 * s + 2);
+          if (2 * s + 3 < it.len) e1n = load_entry(a, it, 2 * s + 3);
           const int j0 = e0 & 0xFFFF, j1 = e1 & 0xFFFF;
           const int kst = g % NK;
           const uint32_t uk = g / NK;
@@ -403,17 +421,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (nblk == 2) tma_load_2d(kdst + c * S::kChunk + 8192, &tmK, 64 * c, row0 + 64 * j1, &k_full[kst]);
           }
           k_phase[kst] = uk & 1;
-          const int vst = g % NV;
-          const uint32_t uv = g / NV;
-          if (uv >= 1 && !mbar_wait(&v_empty[vst], (uv - 1) & 1, abort_flag, a.err, kBackoffNs)) { ok = false; break; }
-          uint8_t* vdst = sm + S::kV + vst * S::kTile;
-          mbar_expect_tx(&v_full[vst], nblk * kTxBlock);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(vdst + c * S::kChunk, &tmV, 64 * c, row0 + 64 * j0, &v_full[vst]);
-            if (nblk == 2) tma_load_2d(vdst + c * S::kChunk + 8192, &tmV, 64 * c, row0 + 64 * j1, &v_full[vst]);
-          }
-          v_phase[vst] = uv & 1;
         }
         ++t;
       }
@@ -421,10 +428,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Drain: let every load this thread issued land before the CTA exits.
         for (int i = 0; i < NK; ++i)
           if (k_phase[i] >= 0) mbar_wait_drain(&k_full[i], k_phase[i], a.err);
-        for (int i = 0; i < NV; ++i)
-          if (v_phase[i] >= 0) mbar_wait_drain(&v_full[i], v_phase[i], a.err);
         for (int b = 0; b < QB; ++b)
           if (q_phase[b] >= 0) mbar_wait_drain(&q_full[b], q_phase[b], a.err);
+      }
+    }
+  } else if (warp == 10) {
+    // ======================= TMA producer: V =======================
+    // A second issuing warp: one thread issues a TMA instruction in about 170
+    // cycles, so Q/K and V come from separate warps, and a V block (all of d)
+    // is one 3D box.
+    if (lane == 0) {
+      uint32_t g = 0;
+      int v_phase[NV];
+      for (int i = 0; i < NV; ++i) v_phase[i] = -1;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int k = item_index(r, cta, G);
+        if (k >= total) break;
+        const Item it = load_item(a, k);
+        const int nsteps = (it.len + 1) >> 1;
+        if (nsteps == 0) continue;
+        const int row0 = it.bh * a.N;
+        uint32_t e0n = load_entry(a, it, 0);
+        uint32_t e1n = it.len > 1 ? load_entry(a, it, 1) : 0u;
+        for (int s = 0; s < nsteps; ++s, ++g) {
+          const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
+          const uint32_t e0 = e0n, e1 = nblk == 2 ? e1n : 0u;
+          if (2 * s + 2 < it.len) e0n = load_entry(a, it, 2 * s + 2);
+          if (2 * s + 3 < it.len) e1n = load_entry(a, it, 2 * s + 3);
+          const int vst = g % NV;
+          const uint32_t uv = g / NV;
+          if (uv >= 1 && !mbar_wait(&v_empty[vst], (uv - 1) & 1, abort_flag, a.err, kBackoffNs)) { ok = false; break; }
+          uint8_t* vdst = sm + S::kV + vst * S::kTile;
+          mbar_expect_tx(&v_full[vst], nblk * kTxBlock);
+          if constexpr (D == 128) {
+            tma_load_3d(vdst, &tmV, 0, row0 + 64 * (e0 & 0xFFFF), 0, &v_full[vst]);
+            if (nblk == 2) tma_load_3d(vdst + S::kVBlock, &tmV, 0, row0 + 64 * (e1 & 0xFFFF), 0, &v_full[vst]);
+          } else {
+            tma_load_2d(vdst, &tmV, 0, row0 + 64 * (e0 & 0xFFFF), &v_full[vst]);
+            if (nblk == 2) tma_load_2d(vdst + S::kVBlock, &tmV, 0, row0 + 64 * (e1 & 0xFFFF), &v_full[vst]);
+          }
+          v_phase[vst] = uv & 1;
+        }
+      }
+      if (!ok || *abort_flag) {
+        for (int i = 0; i < NV; ++i)
+          if (v_phase[i] >= 0) mbar_wait_drain(&v_full[i], v_phase[i], a.err);
       }
     }
   } else if (warp == 1) {
@@ -437,13 +486,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int pnblk = 0;
       auto do_pv = [&]() -> bool {
         const int vst = pg % NV;
-        if (!mbar_wait(&p_full[pg & 1], (pg >> 1) & 1, abort_flag, a.err, kBackoffNs)) return false;
-        if (!mbar_wait(&v_full[vst], (pg / NV) & 1, abort_flag, a.err, kBackoffNs)) return false;
+        if (!mbar_wait(&p_full[pg & 1], (pg >> 1) & 1, abort_flag, a.err)) return false;
+        if (!mbar_wait(&v_full[vst], (pg / NV) & 1, abort_flag, a.err)) return false;
         tc_fence_after();
-        const uint64_t bdesc = smem_desc_sw128(smem_u32(sm + S::kV + vst * S::kTile), S::kChunk, 1024);
-        issue_pv(tm + 256, tm + 384, tm + (pg & 1) * 128, bdesc, idesc_pv, pacc, pnblk);
-        tc_commit(&v_empty[vst]);
-        tc_commit(o_done);
+        const uint32_t vaddr = smem_u32(sm + S::kV + vst * S::kTile);
+        const uint64_t bdesc0 = smem_desc_sw128(vaddr, 64 * 128, 1024);  // LBO: next 64-column chunk of d
+        const uint64_t bdesc1 = smem_desc_sw128(vaddr + S::kVBlock, 64 * 128, 1024);
+        issue_pv(tm + 256, tm + 384, tm + (pg & 1) * 128, bdesc0, bdesc1, idesc_pv, pacc, pnblk);
+        tc_commit(&v_empty[vst]);  // also tells a rescaling softmax warp that PV_pg is complete
         if (plast) tc_commit(o_final);
         return true;
       };
@@ -454,17 +504,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nsteps = (it.len + 1) >> 1;
         if (nsteps == 0) continue;
         const int qb = t % QB;
-        if (!mbar_wait(&q_full[qb], (t / QB) & 1, abort_flag, a.err, kBackoffNs)) { ok = false; break; }
+        if (!mbar_wait(&q_full[qb], (t / QB) & 1, abort_flag, a.err)) { ok = false; break; }
         const uint64_t adesc = smem_desc_sw128(smem_u32(sm + S::kQ + qb * S::kTile), 16, 1024);
         for (int s = 0; s < nsteps; ++s, ++g) {
           const int kst = g % NK;
-          if (!mbar_wait(&k_full[kst], (g / NK) & 1, abort_flag, a.err, kBackoffNs)) { ok = false; break; }
+          if (!mbar_wait(&k_full[kst], (g / NK) & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
           const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
           const uint64_t bdesc = smem_desc_sw128(smem_u32(sm + S::kK + kst * S::kTile), 16, 1024);
           issue_qk<D>(tm + (g & 1) * 128, adesc, bdesc, idesc_bf16_f32(128, 64 * nblk, 0, 0));
-          tc_commit(&s_full[g & 1]);
-          tc_commit(&k_empty[kst]);
+          tc_commit(&s_full[g & 1]);  // K stage kst is released by a softmax warp once S_g is complete
           if (s == nsteps - 1) tc_commit(&q_empty[qb]);
           if (have_pend && !do_pv()) { ok = false; break; }
           have_pend = true;
@@ -531,6 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (2 * s + 2 + cb < it.len) en = load_entry(a, it, 2 * s + 2 + cb);
         if (!warp_wait(&s_full[sb], (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
         tc_fence_after();
+        if (sw == 0 && lane == 0) mbar_arrive(&k_empty[g % NK]);  // S_g done: its K stage is free
         const bool bm = (e >> (16 + half)) & 1u;  // this half's query block selected the key block
         uint32_t pk[32];
         float alpha = 1.f, sum = 0.f;
@@ -566,8 +616,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l = l * alpha + sum;
         if (__any_sync(0xffffffffu, rescale)) {
-          // O_cb holds PV results up to step g-1: wait for PV_{g-1}, then scale.
-          if (!warp_wait(o_done, (g - 1) & 1, abort_flag, a.err)) { ok = false; break; }
+          // O_cb holds PV results up to step g-1: wait for PV_{g-1} (its commit
+          // releases V stage (g-1) % NV; that barrier's earlier phases are
+          // complete because S_g, issued after PV_{g-2}, is), then scale.
+          if (!warp_wait(&v_empty[(g - 1) % NV], ((g - 1) / NV) & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int cc = 0; cc < D; cc += 32) {
@@ -852,6 +904,22 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 // 2D view [rows = B*H*N][d] bf16, 64 x 64 boxes, 128-byte swizzle.
+// 3D view of V for d = 128: (64 columns, rows, 2 chunks of 64 columns), box
+// 64 x 64 x 2, so one TMA instruction moves a whole 64-row block laid out as
+// [chunk][64 rows][128 B] with 128-byte swizzle.
+static bool make_map_v3(CUtensorMap* map, const void* base, size_t rows, int d) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(d / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, 128};
+  cuuint32_t box[3] = {64, 64, static_cast<cuuint32_t>(d / 64)};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 static bool make_map(CUtensorMap* map, const void* base, size_t rows, int d) {
   auto enc = get_encode();
   if (!enc) return false;
@@ -870,8 +938,8 @@ static cudaError_t launch_attn_kernel(const void* Q, const void* K, const void* 
                                       const AttnArgs& args, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
   const size_t rows = static_cast<size_t>(BH) * N;
-  if (!make_map(&mq, Q, rows, D) || !make_map(&mk, K, rows, D) || !make_map(&mv, V, rows, D))
-    return cudaErrorInvalidValue;
+  const bool v_ok = (D == 128) ? make_map_v3(&mv, V, rows, D) : make_map(&mv, V, rows, D);
+  if (!make_map(&mq, Q, rows, D) || !make_map(&mk, K, rows, D) || !v_ok) return cudaErrorInvalidValue;
   DeviceInfo di;
   cudaError_t e = device_info(&di);
   if (e != cudaSuccess) return e;
