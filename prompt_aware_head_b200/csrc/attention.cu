@@ -52,7 +52,7 @@ struct AttnArgs {
   int* err;
 };
 
-constexpr int kThreads = 352;  // Q/K producer, MMA issuer, 8 softmax warps, V producer
+constexpr int kThreads = 384;  // Q/K producer, S issuer, 8 softmax warps, V producer, PV issuer
 constexpr int kNoBlock = 0xFFFF;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t kBackoffNs = 40;            // producer / MMA poll back-off  // log2 units: rescale O when the max grows by > 2^8
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = bars + 4;              // [2]
   uint64_t* p_full = bars + 6;              // [2]
   uint64_t* o_final = bars + 9;             // after the last PV of an item
-  uint64_t* drain = bars + 10;              // abort path
+  uint64_t* drain = bars + 10;              // [2] abort path (one per MMA issuer)
   uint64_t* k_full = bars + 12;             // [NK]
   uint64_t* k_empty = k_full + NK;          // [NK] after the S MMA that read the stage
   uint64_t* v_full = k_empty + NK;          // [NV]
@@ -348,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(o_final, 1);
     mbar_init(drain, 1);
+    mbar_init(drain + 1, 1);
     for (int i = 0; i < NK; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
@@ -477,26 +478,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ======================= MMA issuer =======================
+    // ======================= MMA issuer: S = Q K^T =======================
+    // S and PV are issued by two warps (a thread that issues MMAs blocks while
+    // the tensor core drains them, and one thread doing both serialised the
+    // pipeline).  With two issuers the tensor core no longer orders S after
+    // PV, so S_g waits for PV_{g-2} to complete before overwriting that
+    // S / P buffer: PV_{g-2}'s commit releases V stage (g-2) % NV, and that
+    // barrier's older phases are complete because S_{g-1} waited for PV_{g-3}.
     if (lane == 0) {
-      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
       uint32_t g = 0, t = 0;
-      bool ok = true, have_pend = false;
-      uint32_t pg = 0, pacc = 0, plast = 0;
-      int pnblk = 0;
-      auto do_pv = [&]() -> bool {
-        const int vst = pg % NV;
-        if (!mbar_wait(&p_full[pg & 1], (pg >> 1) & 1, abort_flag, a.err)) return false;
-        if (!mbar_wait(&v_full[vst], (pg / NV) & 1, abort_flag, a.err)) return false;
-        tc_fence_after();
-        const uint32_t vaddr = smem_u32(sm + S::kV + vst * S::kTile);
-        const uint64_t bdesc0 = smem_desc_sw128(vaddr, 64 * 128, 1024);  // LBO: next 64-column chunk of d
-        const uint64_t bdesc1 = smem_desc_sw128(vaddr + S::kVBlock, 64 * 128, 1024);
-        issue_pv(tm + 256, tm + 384, tm + (pg & 1) * 128, bdesc0, bdesc1, idesc_pv, pacc, pnblk);
-        tc_commit(&v_empty[vst]);  // also tells a rescaling softmax warp that PV_pg is complete
-        if (plast) tc_commit(o_final);
-        return true;
-      };
+      bool ok = true;
       for (int r = 0; ok; ++r) {
         const int k = item_index(r, cta, G);
         if (k >= total) break;
@@ -509,26 +500,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < nsteps; ++s, ++g) {
           const int kst = g % NK;
           if (!mbar_wait(&k_full[kst], (g / NK) & 1, abort_flag, a.err)) { ok = false; break; }
+          if (g >= 2 && !mbar_wait(&v_empty[(g - 2) % NV], ((g - 2) / NV) & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
           const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
           const uint64_t bdesc = smem_desc_sw128(smem_u32(sm + S::kK + kst * S::kTile), 16, 1024);
           issue_qk<D>(tm + (g & 1) * 128, adesc, bdesc, idesc_bf16_f32(128, 64 * nblk, 0, 0));
           tc_commit(&s_full[g & 1]);  // K stage kst is released by a softmax warp once S_g is complete
           if (s == nsteps - 1) tc_commit(&q_empty[qb]);
-          if (have_pend && !do_pv()) { ok = false; break; }
-          have_pend = true;
-          pg = g;
-          pnblk = nblk;
-          pacc = s > 0 ? 1u : 0u;
-          plast = (s == nsteps - 1) ? 1u : 0u;
         }
         ++t;
       }
-      if (ok && have_pend && !do_pv()) ok = false;
       if (!ok || *abort_flag) {
         // Drain: wait until every MMA this thread issued has completed.
         tc_commit(drain);
         mbar_wait_drain(drain, 0, a.err);
+      }
+    }
+  } else if (warp == 11) {
+    // ======================= MMA issuer: O_c += P_c V_c =======================
+    if (lane == 0) {
+      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      uint32_t g = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int k = item_index(r, cta, G);
+        if (k >= total) break;
+        const Item it = load_item(a, k);
+        const int nsteps = (it.len + 1) >> 1;
+        if (nsteps == 0) continue;
+        for (int s = 0; s < nsteps; ++s, ++g) {
+          const int vst = g % NV;
+          if (!mbar_wait(&p_full[g & 1], (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
+          if (!mbar_wait(&v_full[vst], (g / NV) & 1, abort_flag, a.err)) { ok = false; break; }
+          tc_fence_after();
+          const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
+          const uint32_t vaddr = smem_u32(sm + S::kV + vst * S::kTile);
+          const uint64_t bdesc0 = smem_desc_sw128(vaddr, 64 * 128, 1024);  // LBO: next 64-column chunk of d
+          const uint64_t bdesc1 = smem_desc_sw128(vaddr + S::kVBlock, 64 * 128, 1024);
+          issue_pv(tm + 256, tm + 384, tm + (g & 1) * 128, bdesc0, bdesc1, idesc_pv, s > 0 ? 1u : 0u, nblk);
+          tc_commit(&v_empty[vst]);  // V stage free; PV_g complete (S_{g+2} and O rescales wait on it)
+          if (s == nsteps - 1) tc_commit(o_final);
+        }
+      }
+      if (!ok || *abort_flag) {
+        tc_commit(drain + 1);
+        mbar_wait_drain(drain + 1, 0, a.err);
       }
     }
   } else {
