@@ -176,7 +176,7 @@ def traffic_from_profile(kernel_src):
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("attention.cu sha256[:16]") != digest:
+    if vals.get("attention.cu sha256 (first 16 hex)") != digest:
         return None
     try:
         return float(vals["dram bytes per launch (full size)"])
