@@ -170,7 +170,9 @@ SA_API sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void*
  * device memory inside the library, which every GPU that loads the library
  * holds until the process exits.  2 * B * H * nB * d * 4 bytes must fit in
  * it (e.g. B1 H24 N33280 d128 needs 12.8 MB); larger calls return
- * SA_ERR_WORKSPACE before anything is launched.  The call allocates nothing.
+ * SA_ERR_WORKSPACE before anything is launched.  When scores_out is NULL the
+ * scores are kept in the same array too, so the heads are then processed in
+ * as many groups as that takes.  The call allocates nothing.
  * The first call on a device looks up the array's device address for that
  * device, so make that first call before any stream capture.  All calls
  * share the one array, which keeps the last call's contents (each call

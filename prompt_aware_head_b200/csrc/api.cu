@@ -20,10 +20,13 @@ WsLayout ws_layout(int B, int H, int N, int d) {
   size_t off = 0;
   w.header = off;
   off += sizeof(WsHeader);
+  const size_t img = (nB + 127) / 128 * 128 * d * sizeof(float);  // one head's operand images (hi or lo)
   w.qbar = off;
-  off += align256(BH * nB * d * sizeof(float));
+  off += align256(2 * BH * img);
   w.kbar = off;
-  off += align256(BH * nB * d * sizeof(float));
+  off += align256(2 * BH * img);
+  w.scores = off;
+  off += align256(BH * nB * nB * sizeof(float));
   w.items = off;
   off += align256(BH * nB * sizeof(int4));
   w.ulist = off;

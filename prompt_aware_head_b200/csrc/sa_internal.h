@@ -24,7 +24,8 @@ namespace sa {
 // Workspace layout (byte offsets from the caller's workspace base).
 struct WsLayout {
   size_t header = 0;        // WsHeader (256 B)
-  size_t qbar = 0, kbar = 0;  // fp32 [BH][nB][d] block means
+  size_t qbar = 0, kbar = 0;  // block means as tf32 hi / lo operand images: [2][BH][row tiles][d/32][128][32]
+  size_t scores = 0;        // fp32 [BH][nB][nB] tile-pair scores (when the caller asks for none)
   size_t items = 0;         // int4 [BH*nB] attention work items (execution order)
   size_t ulist = 0;         // int32 [BH][nB][nB] union lists (j | bits << 16)
   size_t rowbits = 0;       // uint32 [BH][nB][32] per-row block bitmaps
@@ -63,5 +64,6 @@ cudaError_t launch_dense_attention(const void* Q, const void* K, const void* V, 
                                    float scale, void* O, void* ws, cudaStream_t s);
 
 cudaError_t launch_exp2_poly(const float* y, float* out, int n, cudaStream_t s);
+
 
 }  // namespace sa

@@ -15,63 +15,6 @@
 
 namespace sa {
 
-// ============================================================== pooling
-// One CTA per (query/key block i, head bh): mean of the 64 rows of Q and K.
-// 16-byte vector loads, fp32 sums in a fixed order (per-thread rows, then
-// row groups in order), scaled by 1/64 (exact).  HBM-bound.
-template <int D>
-__global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restrict__ Q,
-                                                   const __nv_bfloat16* __restrict__ K, float* __restrict__ qbar,
-                                                   float* __restrict__ kbar, int N, int nB, int H,
-                                                   uint64_t head_bits) {
-  const int i = blockIdx.x, bh = blockIdx.y;
-  if (!((head_bits >> (bh % H)) & 1ull)) return;
-  constexpr int TPR = D / 8;     // threads per row, 8 bf16 (16 B) each
-  constexpr int RG = 128 / TPR;  // row groups
-  constexpr int RPT = 64 / RG;   // rows per thread
-  const int t = threadIdx.x, cg = t % TPR, rg = t / TPR;
-  const size_t base = (static_cast<size_t>(bh) * N + static_cast<size_t>(i) * kBlock) * D;
-  const uint4* q4 = reinterpret_cast<const uint4*>(Q + base);
-  const uint4* k4 = reinterpret_cast<const uint4*>(K + base);
-  uint4 qv[RPT], kv[RPT];
-#pragma unroll
-  for (int r = 0; r < RPT; ++r) {
-    const int row = rg + r * RG;
-    qv[r] = __ldg(q4 + row * TPR + cg);
-    kv[r] = __ldg(k4 + row * TPR + cg);
-  }
-  float aq[8], ak[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) aq[e] = ak[e] = 0.f;
-#pragma unroll
-  for (int r = 0; r < RPT; ++r) {
-    const uint32_t qw[4] = {qv[r].x, qv[r].y, qv[r].z, qv[r].w};
-    const uint32_t kw[4] = {kv[r].x, kv[r].y, kv[r].z, kv[r].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      aq[2 * e] += __uint_as_float(qw[e] << 16);
-      aq[2 * e + 1] += __uint_as_float(qw[e] & 0xFFFF0000u);
-      ak[2 * e] += __uint_as_float(kw[e] << 16);
-      ak[2 * e + 1] += __uint_as_float(kw[e] & 0xFFFF0000u);
-    }
-  }
-  __shared__ float red[2][RG][D];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    red[0][rg][cg * 8 + e] = aq[e];
-    red[1][rg][cg * 8 + e] = ak[e];
-  }
-  __syncthreads();
-  for (int c = t; c < 2 * D; c += 128) {
-    const int which = c / D, col = c % D;
-    float s = 0.f;
-#pragma unroll
-    for (int g = 0; g < RG; ++g) s += red[which][g][col];
-    float* out = which ? kbar : qbar;
-    out[(static_cast<size_t>(bh) * nB + i) * D + col] = s * (1.0f / 64.0f);
-  }
-}
-
 // ============================================================== ranking
 // Order-preserving map of a finite fp32 score to uint32 (larger key = larger
 // score); -0 ranks as +0.
@@ -136,75 +79,497 @@ __device__ __forceinline__ int warp_emit(uint32_t keep, int32_t* out) {
   return base;
 }
 
-// ============================================================== score + select
-// One CTA per (16 query blocks, head).  Scores s_ij = qbar_i . kbar_j in
-// fp32 (CUDA-core FMA, fixed order over d), kept in shared memory; then one
-// warp per row ranks its candidates.
-constexpr int kSelRows = 16;
-constexpr int kKeyChunk = 64;
-
-template <int D, int NC>
-__global__ void __launch_bounds__(256) score_select_kernel(const float* __restrict__ qbar,
-                                                           const float* __restrict__ kbar,
-                                                           const uint8_t* __restrict__ cls, int nB, int H,
-                                                           uint64_t head_bits, int k, int cap,
-                                                           int32_t* __restrict__ idx, int32_t* __restrict__ counts,
-                                                           float* __restrict__ scores_out) {
-  constexpr int R = kSelRows, CH = kKeyChunk, KS = D + 4, SW = NC * 32;
-  extern __shared__ __align__(16) float smem_f[];
-  float* qs = smem_f;         // [R][D]
-  float* ks = qs + R * D;     // [CH][KS]
-  float* sc = ks + CH * KS;   // [R][SW]
-  const int bh = blockIdx.y, i0 = blockIdx.x * R, t = threadIdx.x;
-  if (!((head_bits >> (bh % H)) & 1ull)) {
-    for (int r = t; r < R; r += blockDim.x)
-      if (i0 + r < nB) counts[static_cast<size_t>(bh) * nB + i0 + r] = 0;
-    return;
-  }
-  for (int e = t; e < R * D; e += blockDim.x) {
-    const int r = e / D, c = e % D;
-    qs[e] = (i0 + r < nB) ? qbar[(static_cast<size_t>(bh) * nB + i0 + r) * D + c] : 0.f;
-  }
-  const int r = t >> 4, cl = t & 15;
-  for (int j0 = 0; j0 < nB; j0 += CH) {
-    __syncthreads();
-    for (int e = t; e < CH * (D / 4); e += blockDim.x) {
-      const int row = e / (D / 4), c4 = e % (D / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j0 + row < nB) v = reinterpret_cast<const float4*>(kbar + (static_cast<size_t>(bh) * nB + j0 + row) * D)[c4];
-      *reinterpret_cast<float4*>(ks + row * KS + c4 * 4) = v;
-    }
-    __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const float4* qr = reinterpret_cast<const float4*>(qs + r * D);
-#pragma unroll 8
-    for (int c4 = 0; c4 < D / 4; ++c4) {
-      const float4 a = qr[c4];
+// Top-k over candidate keys by an 8-bit radix select (4 passes, most
+// significant digit first) over a per-warp shared histogram; returns the
+// chosen bits like warp_topk (keys compare by value, ties by lower j).
+template <int NC>
+__device__ __forceinline__ uint32_t warp_topk_radix(const uint32_t (&key)[NC], uint32_t cand, int k,
+                                                    uint32_t* hist) {
+  const int lane = threadIdx.x & 31;
+  const int ncand = __reduce_add_sync(0xffffffffu, __popc(cand));
+  if (k >= ncand) return cand;
+  uint32_t prefix = 0, pmask = 0;
+  int kk = k;  // rank still to place among keys matching the prefix
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4 b = *reinterpret_cast<const float4*>(ks + (cl + 16 * u) * KS + c4 * 4);
-        acc[u] = fmaf(a.x, b.x, acc[u]);
-        acc[u] = fmaf(a.y, b.y, acc[u]);
-        acc[u] = fmaf(a.z, b.z, acc[u]);
-        acc[u] = fmaf(a.w, b.w, acc[u]);
+    for (int b = 0; b < 8; ++b) hist[lane * 8 + b] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+      if (((cand >> c) & 1u) && (key[c] & pmask) == prefix) atomicAdd(&hist[(key[c] >> shift) & 255u], 1u);
+    __syncwarp();
+    // lane l owns digits 255-8l down to 248-8l
+    uint32_t h[8];
+    uint32_t sum = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      h[b] = hist[255 - (lane * 8 + b)];
+      sum += h[b];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint32_t excl = incl - sum;
+    const uint32_t want = static_cast<uint32_t>(kk);
+    const bool here = excl < want && want <= incl;
+    const int leader = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
+    uint32_t digit = 0, above = 0;
+    if (lane == leader) {
+      uint32_t run = excl;
+      bool found = false;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        if (!found && run + h[b] >= want) {
+          digit = 255u - static_cast<uint32_t>(lane * 8 + b);
+          above = run;  // keys with a larger digit under the same prefix
+          found = true;
+        }
+        run += h[b];
       }
     }
+    digit = __shfl_sync(0xffffffffu, digit, leader);
+    above = __shfl_sync(0xffffffffu, above, leader);
+    prefix |= digit << shift;
+    pmask |= 255u << shift;
+    kk -= static_cast<int>(above);
+    __syncwarp();
+  }
+  // prefix is now the k-th largest key: keep keys above it and the first kk equal ones
+  uint32_t sel = 0;
+  int eq_before = 0;
+  const uint32_t lt = lanemask_lt();
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int j = j0 + cl + 16 * u;
-      if (j < nB) sc[r * SW + j] = acc[u];
+  for (int c = 0; c < NC; ++c) {
+    const bool isc = (cand >> c) & 1u;
+    const bool g = isc && key[c] > prefix;
+    const bool e = isc && key[c] == prefix;
+    const uint32_t em = __ballot_sync(0xffffffffu, e);
+    const int rank = eq_before + __popc(em & lt);
+    if (g || (e && rank < kk)) sel |= 1u << c;
+    eq_before += __popc(em);
+  }
+  return sel;
+}
+
+// Top-k (0 < kk < number of candidates) over fp32 scores s[c] at j = 32c +
+// lane, by value then lower j, for finite scores: a 256-bucket histogram on
+// the linear map t = (s - min) * 256 / (max - min), which never puts a
+// larger score in a lower bucket, locates the bucket that holds the kk-th
+// score; buckets above it are kept whole and the boundary bucket is ranked
+// exactly (pairwise when it holds at most 32 scores, else by the radix
+// select).  Non-finite scores or a zero / overflowing range go to the radix
+// select directly, which orders the same way.
+template <int NC>
+__device__ __forceinline__ uint32_t warp_topk_bucket(const float (&s)[NC], uint32_t cand, int kk, uint32_t* hist,
+                                                     uint32_t* memk) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[NC];
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    key[c] = score_key(s[c]);
+    if ((cand >> c) & 1u) {
+      kmin = min(kmin, key[c]);
+      kmax = max(kmax, key[c]);
     }
   }
-  __syncthreads();
-  if (scores_out) {
-    for (int rr = 0; rr < R && i0 + rr < nB; ++rr)
-      for (int j = t; j < nB; j += blockDim.x)
-        scores_out[(static_cast<size_t>(bh) * nB + i0 + rr) * nB + j] = sc[rr * SW + j];
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  // a non-finite score has a key at or beyond those of +-inf
+  const bool bad = kmax >= 0xFF800000u || kmin <= 0x007FFFFFu;
+  // back from keys to the extreme scores (exact; -0 comes back as +0)
+  const float mn = __uint_as_float((kmin & 0x80000000u) ? (kmin & 0x7FFFFFFFu) : ~kmin);
+  const float mx = __uint_as_float((kmax & 0x80000000u) ? (kmax & 0x7FFFFFFFu) : ~kmax);
+  const float range = mx - mn;
+  const float inv = 256.0f / range;
+  if (bad || !(range > 0.0f) || !isfinite(range) || !isfinite(inv)) return warp_topk_radix<NC>(key, cand, kk, hist);
+  int bin[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) bin[c] = min(255, __float2int_rz((s[c] - mn) * inv));
+#pragma unroll
+  for (int b = 0; b < 8; ++b) hist[lane * 8 + b] = 0u;
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    if ((cand >> c) & 1u) atomicAdd(&hist[bin[c]], 1u);
+  __syncwarp();
+  // lane l owns buckets 255-8l down to 248-8l
+  uint32_t h[8], sum = 0;
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    h[b] = hist[255 - (lane * 8 + b)];
+    sum += h[b];
   }
-  const int w = t >> 5, lane = t & 31;
-  for (int rr = w; rr < R; rr += 8) {
-    const int i = i0 + rr;
-    if (i >= nB) break;
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const uint32_t excl = incl - sum, want = static_cast<uint32_t>(kk);
+  const int leader = __ffs(__ballot_sync(0xffffffffu, excl < want && want <= incl)) - 1;
+  int bstar = 0;
+  uint32_t above = 0, m = 0;
+  if (lane == leader) {
+    uint32_t run = excl;
+    bool found = false;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      if (!found && run + h[b] >= want) {
+        bstar = 255 - (lane * 8 + b);
+        above = run;
+        m = h[b];
+        found = true;
+      }
+      run += h[b];
+    }
+  }
+  bstar = __shfl_sync(0xffffffffu, bstar, leader);
+  above = __shfl_sync(0xffffffffu, above, leader);
+  m = __shfl_sync(0xffffffffu, m, leader);
+  const int r = kk - static_cast<int>(above);  // 1..m of the boundary bucket's scores are kept
+  uint32_t sel = 0, inb = 0;
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    if ((cand >> c) & 1u) {
+      if (bin[c] > bstar) sel |= 1u << c;
+      else if (bin[c] == bstar) inb |= 1u << c;
+    }
+  if (r == static_cast<int>(m)) return sel | inb;
+  __syncwarp();
+  if (m > 32u) return sel | warp_topk_radix<NC>(key, inb, r, hist);
+  // members in ascending j: position p holds the p-th one
+  const uint32_t lt = lanemask_lt();
+  int pos[NC];
+  int base = 0;
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const bool in = (inb >> c) & 1u;
+    const uint32_t bm = __ballot_sync(0xffffffffu, in);
+    pos[c] = base + __popc(bm & lt);
+    if (in) memk[pos[c]] = key[c];
+    base += __popc(bm);
+  }
+  __syncwarp();
+  bool win = false;
+  if (lane < static_cast<int>(m)) {
+    const uint32_t kl = memk[lane];
+    int rank = 0;
+    for (int q = 0; q < static_cast<int>(m); ++q) {
+      const uint32_t kq = memk[q];
+      rank += (kq > kl || (kq == kl && q < lane)) ? 1 : 0;
+    }
+    win = rank < r;
+  }
+  const uint32_t wins = __ballot_sync(0xffffffffu, win);
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    if (((inb >> c) & 1u) && ((wins >> pos[c]) & 1u)) sel |= 1u << c;
+  __syncwarp();
+  return sel;
+}
+
+// ============================================================== selection in three kernels
+// The path of sa_select_blocks (and, a group of heads at a time, of
+// sa_select_blocks_noalloc):
+//   pool_kernel      - one CTA per 64-row block of Q and K: their means, each
+//                      split into a tf32 part and the fp32 remainder, written
+//                      straight into the operand images the tensor cores read;
+//   score_tc_kernel  - one CTA per 128 x 256 tile of a head's scores: bulk
+//                      copies of the images, 3xTF32 MMAs into TMEM;
+//   rank_rows_kernel - one warp per row keeps the pins, the diagonal and the
+//                      top k - 1 scores (bucket select).
+// Kernel boundaries order the three, so every image is complete before a
+// tile reads it.
+//
+// Operand images: block means of a head in row tiles of 128 blocks and
+// column chunks of 32 (of d), each a 16 KB image of 128 rows x 128 bytes laid
+// out as the K-major 128-byte-swizzled shared-memory tile the MMA descriptors
+// address: row t at byte 128 t, its 16-byte group g at group g ^ (t & 7).
+// Four arrays (q hi, q lo, k hi, k lo), each [slot][row tile][chunk][128][32].
+// hi = tf32(x) rounded to nearest, lo = x - hi (exact); the MMAs accumulate
+// A_hi B_lo + A_lo B_hi + A_hi B_hi in fp32, which leaves each product within
+// about 2^-22 |a||b| of exact (the dropped lo lo term and the tf32 truncation
+// of lo), as accurate as an fp32 dot product for d <= 128.
+constexpr int kTcM = 128;                 // query blocks per tile (rows of A, TMEM lanes)
+constexpr int kTcN = 256;                 // key blocks per tile (two row tiles of B)
+constexpr int kImgBytes = kTcM * 128;     // one 128-row x 32-fp32 image: 16 KB
+constexpr int kImgFloats = kImgBytes / 4;
+constexpr int kTcStage = 6 * kImgBytes;   // A hi, A lo, B hi (2 tiles), B lo (2 tiles)
+constexpr int kTcSmem = 2 * kTcStage + 1024 + 128;
+
+// Instruction descriptor: kind::tf32 with tf32 A/B (both K-major), fp32 D.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ float tf32_rn(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+// Float offset of block i, dimension col inside a head's image array.
+template <int D>
+__device__ __forceinline__ size_t img_offset(int i, int col) {
+  const int rt = i >> 7, t = i & 127, kc = col >> 5, g = (col & 31) >> 2;
+  return (static_cast<size_t>(rt) * (D / 32) + kc) * kImgFloats + t * 32 + ((g ^ (t & 7)) << 2) + (col & 3);
+}
+
+// One CTA per (query/key block i, head bh = bh0 + slot): mean of the 64 rows
+// of Q and K.  16-byte vector loads, fp32 sums in a fixed order (per-thread
+// rows, then row groups in order), scaled by 1/64 (exact), then split into
+// hi / lo and written to the images of slot (RT row tiles per head).
+// HBM-bound.
+template <int D>
+__global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                   const __nv_bfloat16* __restrict__ K, float* __restrict__ qimg,
+                                                   float* __restrict__ kimg, int N, int nB, int RT, int H,
+                                                   uint64_t head_bits, int bh0, size_t lo_offset) {
+  const int i = blockIdx.x, slot = blockIdx.y, bh = bh0 + slot;
+  if (!((head_bits >> (bh % H)) & 1ull)) return;
+  constexpr int TPR = D / 8;     // threads per row, 8 bf16 (16 B) each
+  constexpr int RG = 128 / TPR;  // row groups
+  constexpr int RPT = 64 / RG;   // rows per thread
+  const int t = threadIdx.x, cg = t % TPR, rg = t / TPR;
+  const size_t base = (static_cast<size_t>(bh) * N + static_cast<size_t>(i) * kBlock) * D;
+  const uint4* q4 = reinterpret_cast<const uint4*>(Q + base);
+  const uint4* k4 = reinterpret_cast<const uint4*>(K + base);
+  uint4 qv[RPT], kv[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const int row = rg + r * RG;
+    qv[r] = __ldg(q4 + row * TPR + cg);
+    kv[r] = __ldg(k4 + row * TPR + cg);
+  }
+  float aq[8], ak[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) aq[e] = ak[e] = 0.f;
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const uint32_t qw[4] = {qv[r].x, qv[r].y, qv[r].z, qv[r].w};
+    const uint32_t kw[4] = {kv[r].x, kv[r].y, kv[r].z, kv[r].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      aq[2 * e] += __uint_as_float(qw[e] << 16);
+      aq[2 * e + 1] += __uint_as_float(qw[e] & 0xFFFF0000u);
+      ak[2 * e] += __uint_as_float(kw[e] << 16);
+      ak[2 * e + 1] += __uint_as_float(kw[e] & 0xFFFF0000u);
+    }
+  }
+  __shared__ float red[2][RG][D];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    red[0][rg][cg * 8 + e] = aq[e];
+    red[1][rg][cg * 8 + e] = ak[e];
+  }
+  __syncthreads();
+  const size_t head = static_cast<size_t>(slot) * RT * (D / 32) * kImgFloats;
+  for (int c = t; c < 2 * D; c += 128) {
+    const int which = c / D, col = c % D;
+    float s = 0.f;
+#pragma unroll
+    for (int g = 0; g < RG; ++g) s += red[which][g][col];
+    s *= (1.0f / 64.0f);
+    const float hi = tf32_rn(s);
+    float* img = (which ? kimg : qimg) + head + img_offset<D>(i, col);
+    img[0] = hi;
+    img[lo_offset] = s - hi;
+  }
+}
+
+struct TcArgs {
+  const float* qimg;  // q hi images; q lo at + lo_offset
+  const float* kimg;  // k hi images; k lo at + lo_offset
+  float* scores;      // [slot][nB][nB]
+  int* err;
+  size_t lo_offset;
+  int nB, RT, H, bh0;
+  uint64_t head_bits;
+};
+
+// The 12 MMAs of one 32-wide chunk of d: 4 steps of K = 8, each adding
+// A_hi B_lo, A_lo B_hi and A_hi B_hi (the small terms first) into D.
+__device__ __forceinline__ void tc_issue_chunk(uint32_t d_tmem, uint64_t ahi, uint64_t alo, uint64_t bhi, uint64_t blo,
+                                               uint32_t idesc, int accumulate) {
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const uint64_t o = 2 * s;  // 32 bytes per K = 8 step, in descriptor units
+    asm volatile(
+        "{\n .reg .pred p0, p1;\n setp.ne.b32 p0, %6, 0;\n setp.eq.b32 p1, 0, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %4, %5, p0;\n"
+        " tcgen05.mma.cta_group::1.kind::tf32 [%0], %2, %3, %5, p1;\n"
+        " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %3, %5, p1;\n}\n" ::"r"(d_tmem),
+        "l"(ahi + o), "l"(alo + o), "l"(bhi + o), "l"(blo + o), "r"(idesc), "r"((accumulate || s > 0) ? 1 : 0)
+        : "memory");
+  }
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// One CTA (4 warps) per 128 x 256 tile of one head's scores: query blocks
+// m0 = 128 blockIdx.y + r (row tile blockIdx.y of A), key blocks
+// n0 = 256 blockIdx.x + c (row tiles 2 blockIdx.x and 2 blockIdx.x + 1 of B).
+// Thread 0 streams the d chunks' images through two stages with bulk copies
+// and issues each chunk's MMAs once its stage is full; the MMA commit frees
+// the stage.  Warp w then reads TMEM lanes 32 w .. 32 w + 31 (tile rows) and
+// writes its rows' scores.  Image rows past nB hold whatever was there: they
+// only reach scores that are never written out.
+template <int D>
+__global__ void __launch_bounds__(128, 1) score_tc_kernel(const __grid_constant__ TcArgs a) {
+  constexpr int NKC = D / 32;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + 2 * kTcStage);  // [2]
+  uint64_t* empty = full + 2;                                         // [2]
+  uint64_t* done = empty + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  int* flags = reinterpret_cast<int*>(tslot + 1);
+  volatile int* abort_flag = flags;
+  const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+  const int slot = blockIdx.z, bh = a.bh0 + slot, nB = a.nB, RT = a.RT;
+  if (!((a.head_bits >> (bh % a.H)) & 1ull)) return;
+  const int rt = blockIdx.y, bt0 = 2 * blockIdx.x, nbt = (bt0 + 1 < RT) ? 2 : 1;
+  const int m0 = rt * kTcM, n0 = blockIdx.x * kTcN;
+  if (t == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    flags[0] = 0;
+    mbar_fence_init();
+  }
+  if (w == 0) tmem_alloc(tslot, kTcN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  bool ok = true;
+  if (t == 0) {
+    const size_t head = static_cast<size_t>(slot) * RT * NKC * kImgFloats;
+    const float* qh = a.qimg + head;
+    const float* kh = a.kimg + head;
+    const uint32_t bytes = static_cast<uint32_t>((2 + 2 * nbt) * kImgBytes);
+    auto load = [&](int kc, int s) {
+      unsigned char* st = sm + s * kTcStage;
+      mbar_expect_tx(&full[s], bytes);
+      const size_t ao = (static_cast<size_t>(rt) * NKC + kc) * kImgFloats;
+      bulk_load(st, qh + ao, kImgBytes, &full[s]);
+      bulk_load(st + kImgBytes, qh + a.lo_offset + ao, kImgBytes, &full[s]);
+      for (int b = 0; b < nbt; ++b) {
+        const size_t bo = (static_cast<size_t>(bt0 + b) * NKC + kc) * kImgFloats;
+        bulk_load(st + (2 + b) * kImgBytes, kh + bo, kImgBytes, &full[s]);
+        bulk_load(st + (4 + b) * kImgBytes, kh + a.lo_offset + bo, kImgBytes, &full[s]);
+      }
+    };
+    constexpr uint32_t kIdesc = idesc_tf32_f32(kTcM, kTcN);
+    int loaded = 0, multiplied = 0;
+    load(0, 0);
+    ++loaded;
+    if (NKC > 1) {
+      load(1, 1);
+      ++loaded;
+    }
+    for (int kc = 0; kc < NKC; ++kc) {
+      const int s = kc & 1;
+      if (!mbar_wait(&full[s], (kc >> 1) & 1, abort_flag, a.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t st = smem_u32(sm + s * kTcStage);
+      tc_issue_chunk(tmem, smem_desc_sw128(st, 16, 1024), smem_desc_sw128(st + kImgBytes, 16, 1024),
+                     smem_desc_sw128(st + 2 * kImgBytes, 16, 1024), smem_desc_sw128(st + 4 * kImgBytes, 16, 1024),
+                     kIdesc, kc);
+      tc_commit(&empty[s]);
+      ++multiplied;
+      if (kc + 2 < NKC) {
+        if (!mbar_wait(&empty[s], (kc >> 1) & 1, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        load(kc + 2, s);
+        ++loaded;
+      }
+    }
+    if (ok) {
+      tc_commit(done);
+    } else {  // after an abort: copies and MMAs in flight finish before the CTA leaves
+      for (int x = multiplied; x < loaded; ++x) mbar_wait_drain(&full[x & 1], (x >> 1) & 1, a.err);
+      if (multiplied > 0) mbar_wait_drain(&empty[(multiplied - 1) & 1], ((multiplied - 1) >> 1) & 1, a.err);
+      *abort_flag = 1;
+    }
+  }
+  ok = __syncthreads_and(ok ? 1 : 0) != 0;
+  if (ok) ok = __syncthreads_and(mbar_wait(done, 0, abort_flag, a.err) ? 1 : 0) != 0;
+  tc_fence_after();
+  if (ok) {
+    const int i = m0 + 32 * w + lane;
+    float* out = a.scores + (static_cast<size_t>(slot) * nB + i) * nB;
+#pragma unroll 1
+    for (int cb = 0; cb < kTcN / 32; ++cb) {
+      const int j0 = n0 + 32 * cb;
+      if (j0 >= nB) break;
+      uint32_t r[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * w) << 16) + 32 * cb, r);
+      tmem_wait_ld();
+      if (i < nB) {
+        if ((nB & 3) == 0 && j0 + 32 <= nB) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(out + j0 + c) = make_float4(
+                __uint_as_float(r[c]), __uint_as_float(r[c + 1]), __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (j0 + c < nB) out[j0 + c] = __uint_as_float(r[c]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (w == 0) tmem_dealloc(tmem, kTcN);
+}
+
+// ============================================================== ranking rows
+// One warp per query block row (head bh = bh0 + slot) of the scores
+// score_tc_kernel wrote ([slot][nB][nB]): the pins,
+// the diagonal (it outranks every score) and the top k - 1 other sparse
+// candidates by the bucket select; the list goes out in ascending order.
+// Rows of skipped heads get empty lists.
+template <int NC>
+__global__ void __launch_bounds__(128, 8) rank_rows_kernel(const float* __restrict__ scores,
+                                                           const uint8_t* __restrict__ cls_g, int nB, int H,
+                                                           uint64_t head_bits, int k, int cap,
+                                                           int32_t* __restrict__ idx, int32_t* __restrict__ counts,
+                                                           int bh0) {
+  __shared__ uint32_t hist[4][256];
+  __shared__ uint32_t memk[4][32];
+  __shared__ uint8_t cls[32 * NC];
+  for (int j = threadIdx.x; j < nB; j += 128) cls[j] = cls_g[j];
+  __syncthreads();
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, slot = blockIdx.y, bh = bh0 + slot;
+  const bool active_head = (head_bits >> (bh % H)) & 1ull;
+  for (int rr = 0; rr < 2; ++rr) {  // two rows per warp: one wave covers every row
+    const int i = blockIdx.x * 8 + rr * 4 + w;
+    if (i >= nB) return;
+    const size_t row = static_cast<size_t>(bh) * nB + i;
+    if (!active_head) {
+      if (lane == 0) counts[row] = 0;
+      continue;
+    }
     const uint8_t ci = cls[i];
     uint32_t keep = 0;
     if (ci == kPin) {
@@ -214,26 +579,36 @@ __global__ void __launch_bounds__(256) score_select_kernel(const float* __restri
         if (j < nB && cls[j] != kDrop) keep |= 1u << c;
       }
     } else if (ci == kSparse) {
-      uint32_t key[NC];
-      uint32_t cand = 0, pin = 0;
+      float sc[NC];
+      uint32_t cand = 0, diag = 0;
 #pragma unroll
       for (int c = 0; c < NC; ++c) {
         const int j = 32 * c + lane;
-        key[c] = 0;
+        sc[c] = 0.f;
         if (j < nB) {
           const uint8_t cj = cls[j];
           if (cj == kPin) {
-            pin |= 1u << c;
+            keep |= 1u << c;
           } else if (cj == kSparse) {
-            key[c] = (j == i) ? 0xFFFFFFFFu : score_key(sc[rr * SW + j]);
-            cand |= 1u << c;
+            if (j == i) {
+              diag |= 1u << c;
+            } else {
+              cand |= 1u << c;
+              sc[c] = __ldg(scores + (static_cast<size_t>(slot) * nB + i) * nB + j);
+            }
           }
         }
       }
-      keep = warp_topk<NC>(key, cand, k) | pin;
+      if (k >= 1) {
+        keep |= diag;
+        const int kk = k - 1;
+        const int ncand = __reduce_add_sync(0xffffffffu, __popc(cand));
+        if (kk >= ncand) keep |= cand;
+        else if (kk > 0) keep |= warp_topk_bucket<NC>(sc, cand, kk, hist[w], memk[w]);
+      }
     }
-    const int n = warp_emit<NC>(keep, idx + (static_cast<size_t>(bh) * nB + i) * cap);
-    if (lane == 0) counts[static_cast<size_t>(bh) * nB + i] = n;
+    const int n = warp_emit<NC>(keep, idx + row * cap);
+    if (lane == 0) counts[row] = n;
   }
 }
 
@@ -333,72 +708,103 @@ static int chunks_for(int nB) {
   return -1;
 }
 
-template <int D, int NC>
-static cudaError_t launch_score_select_t(const float* qbar, const float* kbar, const sa_layout* L, int BH, int H,
-                                         uint64_t head_bits, int k, int32_t* idx, int32_t* counts,
-                                         float* scores_out, cudaStream_t s) {
-  constexpr size_t smem = (kSelRows * D + kKeyChunk * (D + 4) + kSelRows * NC * 32) * sizeof(float);
-  static int configured_dev_mask = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!(configured_dev_mask & (1 << (dev & 31)))) {
-    cudaError_t e = cudaFuncSetAttribute(score_select_kernel<D, NC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    configured_dev_mask |= 1 << (dev & 31);
-  }
-  dim3 grid((L->nB + kSelRows - 1) / kSelRows, BH);
-  score_select_kernel<D, NC><<<grid, 256, smem, s>>>(qbar, kbar, L->d_cls, L->nB, H, head_bits, k, L->cap, idx,
-                                                     counts, scores_out);
+// Chunk counts (32 key blocks each) the rank kernel is built for.
+static int select_chunks(int nB) {
+  const int need = (nB + 31) / 32;
+  const int opts[] = {2, 4, 8, 9, 12, 17, 24, 32};
+  for (int o : opts)
+    if (need <= o) return o;
+  return -1;
+}
+
+// Per-device one-time setup of a kernel's dynamic shared memory limit.
+template <typename F>
+static cudaError_t ensure_smem(F* kernel, size_t bytes, bool* configured, std::mutex& mu, int dev) {
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 64 && configured[dev]) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess && dev < 64) configured[dev] = true;
+  return e;
+}
+
+template <int NC>
+static cudaError_t launch_rank_t(const float* scores, const sa_layout* L, int bh0, int nbh, int H, uint64_t head_bits,
+                                 int k, int32_t* idx, int32_t* counts, cudaStream_t s) {
+  rank_rows_kernel<NC><<<dim3((L->nB + 7) / 8, nbh), 128, 0, s>>>(scores, L->d_cls, L->nB, H, head_bits, k, L->cap,
+                                                                 idx, counts, bh0);
   return cudaGetLastError();
 }
 
-template <int D>
-static cudaError_t launch_score_select_d(int nc, const float* qbar, const float* kbar, const sa_layout* L, int BH,
-                                         int H, uint64_t head_bits, int k, int32_t* idx, int32_t* counts,
-                                         float* scores_out, cudaStream_t s) {
+static cudaError_t launch_rank(int nc, const float* scores, const sa_layout* L, int bh0, int nbh, int H,
+                               uint64_t head_bits, int k, int32_t* idx, int32_t* counts, cudaStream_t s) {
   switch (nc) {
-    case 2: return launch_score_select_t<D, 2>(qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
-    case 4: return launch_score_select_t<D, 4>(qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
-    case 8: return launch_score_select_t<D, 8>(qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
-    case 12: return launch_score_select_t<D, 12>(qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
-    case 17: return launch_score_select_t<D, 17>(qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
-    case 24: return launch_score_select_t<D, 24>(qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
-    case 32: return launch_score_select_t<D, 32>(qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
+    case 2: return launch_rank_t<2>(scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
+    case 4: return launch_rank_t<4>(scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
+    case 8: return launch_rank_t<8>(scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
+    case 9: return launch_rank_t<9>(scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
+    case 12: return launch_rank_t<12>(scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
+    case 17: return launch_rank_t<17>(scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
+    case 24: return launch_rank_t<24>(scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
+    case 32: return launch_rank_t<32>(scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// Floats of one head's image array (hi or lo).
+static size_t img_floats(int nB, int d) { return static_cast<size_t>((nB + kTcM - 1) / kTcM) * d * kTcM; }
+
+// The three kernels over heads bh0 .. bh0 + nbh - 1: the images (q, k: hi
+// then lo, nbh heads each) and scores are slot-indexed ([bh - bh0] ...),
+// idx / counts indexed by bh.
+static cudaError_t select_heads(const sa_layout* L, const void* Q, const void* K, int H, int d, int k,
+                                uint64_t head_bits, int bh0, int nbh, float* qimg, float* kimg, float* scores, int* err,
+                                int32_t* idx, int32_t* counts, cudaStream_t s) {
+  static bool configured[2][64];  // per head size, per device
+  static std::mutex mu;
+  const int nB = L->nB, nc = select_chunks(nB), RT = (nB + kTcM - 1) / kTcM;
+  if (nc < 0) return cudaErrorInvalidValue;
+  DeviceInfo di;
+  cudaError_t e = device_info(&di);
+  if (e != cudaSuccess) return e;
+  e = d == 128 ? ensure_smem(score_tc_kernel<128>, kTcSmem, configured[0], mu, di.id)
+               : ensure_smem(score_tc_kernel<64>, kTcSmem, configured[1], mu, di.id);
+  if (e != cudaSuccess) return e;
+  const size_t lo = static_cast<size_t>(nbh) * img_floats(nB, d);
+  const auto* q = static_cast<const __nv_bfloat16*>(Q);
+  const auto* kk = static_cast<const __nv_bfloat16*>(K);
+  if (d == 128)
+    pool_kernel<128><<<dim3(nB, nbh), 128, 0, s>>>(q, kk, qimg, kimg, L->N, nB, RT, H, head_bits, bh0, lo);
+  else
+    pool_kernel<64><<<dim3(nB, nbh), 128, 0, s>>>(q, kk, qimg, kimg, L->N, nB, RT, H, head_bits, bh0, lo);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  TcArgs ta{qimg, kimg, scores, err, lo, nB, RT, H, bh0, head_bits};
+  const dim3 grid((nB + kTcN - 1) / kTcN, RT, nbh);
+  if (d == 128) score_tc_kernel<128><<<grid, 128, kTcSmem, s>>>(ta);
+  else score_tc_kernel<64><<<grid, 128, kTcSmem, s>>>(ta);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return launch_rank(nc, scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
 }
 
 cudaError_t launch_select(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, int k,
                           uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out, void* ws,
                           cudaStream_t s) {
-  const int BH = B * H, nB = L->nB;
-  const int nc = chunks_for(nB);
-  if (nc < 0) return cudaErrorInvalidValue;
   if (k >= L->n_cand && scores_out == nullptr)  // the budget covers every candidate: dense lists, no scoring
     return launch_pattern(L, 3, 0, 0, 1, k, B, H, head_bits, idx, counts, s);
   const WsLayout wl = ws_layout(B, H, L->N, d);
-  float* qbar = reinterpret_cast<float*>(static_cast<char*>(ws) + wl.qbar);
-  float* kbar = reinterpret_cast<float*>(static_cast<char*>(ws) + wl.kbar);
-  dim3 pgrid(nB, BH);
-  if (d == 128)
-    pool_kernel<128><<<pgrid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
-                                           qbar, kbar, L->N, nB, H, head_bits);
-  else
-    pool_kernel<64><<<pgrid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
-                                          qbar, kbar, L->N, nB, H, head_bits);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  if (d == 128) return launch_score_select_d<128>(nc, qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
-  return launch_score_select_d<64>(nc, qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
+  char* base = static_cast<char*>(ws);
+  float* scores = scores_out ? scores_out : reinterpret_cast<float*>(base + wl.scores);
+  return select_heads(L, Q, K, H, d, k, head_bits, 0, B * H, reinterpret_cast<float*>(base + wl.qbar),
+                      reinterpret_cast<float*>(base + wl.kbar), scores,
+                      &reinterpret_cast<WsHeader*>(base + wl.header)->err, idx, counts, s);
 }
 
 // ============================================================== selection without allocation
 // For callers that cannot allocate device memory (see sa_select_blocks_noalloc
-// in sa.h): the pooled block means live in this fixed, file-scope device
-// array instead of the caller's workspace.  Every process that loads the
+// in sa.h): the pooled block means (and the scores when the caller takes
+// none) live in this fixed, file-scope device array instead of the caller's
+// workspace, a group of heads at a time.  Every process that loads the
 // library holds it on every GPU it uses until exit.
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB: q-bar and k-bar, fp32
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB: q-bar, k-bar (and scores), fp32
 static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
 
 size_t select_noalloc_limit() { return kNoAllocScratchBytes; }
@@ -428,28 +834,31 @@ cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void*
                                   uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out,
                                   cudaStream_t s) {
   const int BH = B * H, nB = L->nB;
-  const int nc = chunks_for(nB);
-  if (nc < 0) return cudaErrorInvalidValue;
   if (k >= L->n_cand && scores_out == nullptr)  // dense lists: no scratch used
     return launch_pattern(L, 3, 0, 0, 1, k, B, H, head_bits, idx, counts, s);
   void* scratch = nullptr;
   cudaError_t e = noalloc_scratch(&scratch);
   if (e != cudaSuccess) return e;
-  // q-bar and k-bar are written in full for every active head by the pooling
-  // kernel before the scoring kernel reads them: nothing needs clearing.
-  float* qbar = static_cast<float*>(scratch);
-  float* kbar = qbar + static_cast<size_t>(BH) * nB * d;
-  dim3 pgrid(nB, BH);
-  if (d == 128)
-    pool_kernel<128><<<pgrid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
-                                           qbar, kbar, L->N, nB, H, head_bits);
-  else
-    pool_kernel<64><<<pgrid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
-                                          qbar, kbar, L->N, nB, H, head_bits);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  if (d == 128) return launch_score_select_d<128>(nc, qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
-  return launch_score_select_d<64>(nc, qbar, kbar, L, BH, H, head_bits, k, idx, counts, scores_out, s);
+  // Per group of G heads: the q and k operand images (hi and lo) and (unless
+  // the caller takes them) the scores, then a word for the kernels' error
+  // bits.  Every value that reaches an output is written for each active head
+  // before it is read: nothing needs clearing.
+  const size_t img = img_floats(nB, d) * sizeof(float);  // one head's hi (or lo) images
+  const size_t per_head = 4 * img + (scores_out ? 0 : static_cast<size_t>(nB) * nB * sizeof(float));
+  const int G = static_cast<int>(std::min<size_t>(BH, (kNoAllocScratchBytes - 256) / per_head));
+  if (G < 1) return cudaErrorInvalidValue;
+  char* base = static_cast<char*>(scratch);
+  float* qimg = reinterpret_cast<float*>(base);
+  float* kimg = reinterpret_cast<float*>(base + 2 * G * img);
+  float* sc_scratch = reinterpret_cast<float*>(base + 4 * G * img);
+  int* err = reinterpret_cast<int*>(base + kNoAllocScratchBytes - 256);
+  for (int bh0 = 0; bh0 < BH; bh0 += G) {
+    const int nbh = std::min(G, BH - bh0);
+    float* sc = scores_out ? scores_out + static_cast<size_t>(bh0) * nB * nB : sc_scratch;
+    e = select_heads(L, Q, K, H, d, k, head_bits, bh0, nbh, qimg, kimg, sc, err, idx, counts, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 template <int NC>
