@@ -550,7 +550,7 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(const __grid_constant_
 // candidates by the bucket select; the list goes out in ascending order.
 // Rows of skipped heads get empty lists.
 template <int NC>
-__global__ void __launch_bounds__(128, 8) rank_rows_kernel(const float* __restrict__ scores,
+__global__ void __launch_bounds__(128, NC <= 17 ? 8 : 4) rank_rows_kernel(const float* __restrict__ scores,
                                                            const uint8_t* __restrict__ cls_g, int nB, int H,
                                                            uint64_t head_bits, int k, int cap,
                                                            int32_t* __restrict__ idx, int32_t* __restrict__ counts,
@@ -558,9 +558,21 @@ __global__ void __launch_bounds__(128, 8) rank_rows_kernel(const float* __restri
   __shared__ uint32_t hist[4][256];
   __shared__ uint32_t memk[4][32];
   __shared__ uint8_t cls[32 * NC];
+  __shared__ uint32_t pin_m[NC], sparse_m[NC], drop_m[NC];  // class masks of key blocks 32c + lane
   for (int j = threadIdx.x; j < nB; j += 128) cls[j] = cls_g[j];
   __syncthreads();
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, slot = blockIdx.y, bh = bh0 + slot;
+  for (int c = w; c < NC; c += 4) {
+    const int j = 32 * c + lane;
+    const uint8_t cj = j < nB ? cls[j] : static_cast<uint8_t>(kDrop);
+    const uint32_t pm = __ballot_sync(0xffffffffu, cj == kPin), sm = __ballot_sync(0xffffffffu, cj == kSparse);
+    if (lane == 0) {
+      pin_m[c] = pm;
+      sparse_m[c] = sm;
+      drop_m[c] = ~(pm | sm);
+    }
+  }
+  __syncthreads();
   const bool active_head = (head_bits >> (bh % H)) & 1ull;
   for (int rr = 0; rr < 2; ++rr) {  // two rows per warp: one wave covers every row
     const int i = blockIdx.x * 8 + rr * 4 + w;
@@ -574,30 +586,19 @@ __global__ void __launch_bounds__(128, 8) rank_rows_kernel(const float* __restri
     uint32_t keep = 0;
     if (ci == kPin) {
 #pragma unroll
-      for (int c = 0; c < NC; ++c) {
-        const int j = 32 * c + lane;
-        if (j < nB && cls[j] != kDrop) keep |= 1u << c;
-      }
+      for (int c = 0; c < NC; ++c) keep |= ((~drop_m[c] >> lane) & 1u) << c;
     } else if (ci == kSparse) {
       float sc[NC];
       uint32_t cand = 0, diag = 0;
+      const float* srow = scores + (static_cast<size_t>(slot) * nB + i) * nB + lane;
 #pragma unroll
       for (int c = 0; c < NC; ++c) {
-        const int j = 32 * c + lane;
-        sc[c] = 0.f;
-        if (j < nB) {
-          const uint8_t cj = cls[j];
-          if (cj == kPin) {
-            keep |= 1u << c;
-          } else if (cj == kSparse) {
-            if (j == i) {
-              diag |= 1u << c;
-            } else {
-              cand |= 1u << c;
-              sc[c] = __ldg(scores + (static_cast<size_t>(slot) * nB + i) * nB + j);
-            }
-          }
-        }
+        keep |= ((pin_m[c] >> lane) & 1u) << c;
+        const bool sp = (sparse_m[c] >> lane) & 1u;
+        const bool dg = 32 * c + lane == i;
+        diag |= (sp && dg ? 1u : 0u) << c;
+        cand |= (sp && !dg ? 1u : 0u) << c;
+        sc[c] = (sp && !dg) ? __ldg(srow + 32 * c) : 0.f;
       }
       if (k >= 1) {
         keep |= diag;
