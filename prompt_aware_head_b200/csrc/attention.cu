@@ -22,8 +22,9 @@
 //    O += P V is one asm block of TS MMAs (A from TMEM).  S is double
 //    buffered in TMEM so the MMAs of step g+1 overlap the softmax of step g.
 //  * Warp roles: warp 0 TMA producer for Q and K, warp 10 TMA producer for V,
-//    warp 1 MMA issuer (one thread), warps 2-9 softmax / correction /
-//    epilogue (two warps per tile row, one per key block of a step).
+//    warp 1 issues the S MMAs and warp 11 the PV MMAs (one thread each),
+//    warps 2-9 softmax / correction / epilogue (two warps per tile row, one
+//    per key block of a step).
 //  * Rescaling of O (in TMEM) happens only when a row's running max grows by
 //    more than 2^8; otherwise the stale max is kept (exact after the final
 //    division by the running sum).
