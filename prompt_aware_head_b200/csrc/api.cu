@@ -30,13 +30,11 @@ WsLayout ws_layout(int B, int H, int N, int d) {
   w.items = off;
   off += align256(BH * nB * sizeof(int4));
   w.ulist = off;
-  off += align256(BH * nB * nB * sizeof(int32_t));
-  w.rowbits = off;
-  off += align256(BH * nB * (kMaxBlocks / 32) * sizeof(uint32_t));
+  off += align256(3 * BH * nB * nB * sizeof(int32_t));
   w.lens = off;
-  off += align256(BH * nB * sizeof(int32_t));
+  off += align256(3 * BH * nB * sizeof(int32_t));
   w.totals = off;
-  off += align256(BH * 3 * sizeof(int32_t));
+  off += align256(BH * ((nB + 7) / 8) * 3 * sizeof(int32_t));
   w.total = off;
   return w;
 }
@@ -346,6 +344,8 @@ sa_status sa_attention_plan(const int32_t* idx, const int32_t* counts, int B, in
   if (!idx || !counts) return SA_ERR_INVALID_ARG;
   if (B <= 0 || (d != 64 && d != 128) || N <= 0 || N % kBlock || N / kBlock > kMaxBlocks) return SA_ERR_SHAPE;
   if (cap < 1 || cap > N / kBlock) return SA_ERR_SHAPE;
+  // union lists of all three pairing strides are addressed with int32 offsets
+  if (3ll * B * H * (N / kBlock) * (N / kBlock) >= (1ll << 31)) return SA_ERR_SHAPE;
   uint64_t bits = 0;
   sa_status st = head_bits_of(head_mask, H, min_active, &bits);
   if (st != SA_OK) return st;

@@ -27,10 +27,9 @@ struct WsLayout {
   size_t qbar = 0, kbar = 0;  // block means as tf32 hi / lo operand images: [2][BH][row tiles][d/32][128][32]
   size_t scores = 0;        // fp32 [BH][nB][nB] tile-pair scores (when the caller asks for none)
   size_t items = 0;         // int4 [BH*nB] attention work items (execution order)
-  size_t ulist = 0;         // int32 [BH][nB][nB] union lists (j | bits << 16)
-  size_t rowbits = 0;       // uint32 [BH][nB][32] per-row block bitmaps
-  size_t lens = 0;          // int32 [BH][nB] union length per first block of a pair (-1: not a first)
-  size_t totals = 0;        // int32 [BH][3] summed union length per pairing stride
+  size_t ulist = 0;         // int32 [3 strides][BH][nB][nB] union lists (j | bits << 16)
+  size_t lens = 0;          // int32 [3 strides][BH][nB] union length per first block of a pair (-1: not a first)
+  size_t totals = 0;        // int32 [BH][nB/8 rounded up][3] per-CTA partial sums of union lengths
   size_t total = 0;
 };
 WsLayout ws_layout(int B, int H, int N, int d);
