@@ -222,10 +222,19 @@ def run_ours(args):
     dense_short = k_budget >= L.n_cand
     n_masked = int(H - mask.sum())
 
+    def select(q, k):
+        if args.pattern == "content":
+            sa.sa_select_blocks(L, q, k, B, H, d, rho, mask, w.min_active, idx, counts, None, ws, ws_bytes, stream)
+        elif args.pattern == "radial":
+            sa.sa_pattern_mask(L, sa.SA_PAT_RADIAL, B, H, rho, mask, w.min_active, idx, counts, stream=stream)
+        else:
+            sa.sa_pattern_mask(L, sa.SA_PAT_WINDOW_GLOBAL, B, H, rho, mask, w.min_active, idx, counts,
+                               window_tokens=512, n_global_blocks=8, stream=stream)
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        sa.sa_select_blocks(L, Q, K, B, H, d, rho, mask, w.min_active, idx, counts, None, ws, ws_bytes, stream)
+        select(Q, K)
         if ev is not None:
             ev[1].record(stream)
         sa.sa_attention_plan(idx, counts, B, H, N, d, L.cap, mask, w.min_active, ws, ws_bytes, stream)
@@ -235,7 +244,10 @@ def run_ours(args):
         if ev is not None:
             ev[3].record(stream)
 
-    launches_per_step = (1 if dense_short else 2) + 2 + 1 + (1 if n_masked else 0)
+    # selection (pool, scores, rank; one kernel for a pattern or a budget that
+    # covers every candidate), planner (rows, order), attention (+ zeroing of
+    # skipped heads)
+    launches_per_step = (1 if dense_short or args.pattern != "content" else 3) + 2 + 1 + (1 if n_masked else 0)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -333,7 +345,7 @@ def run_ours(args):
         stream.wait_event(in_done[i])
         if i >= 2:
             stream.wait_event(out_done[i - 2])
-        sa.sa_select_blocks(L, q, k, B, H, d, rho, mask, w.min_active, idx, counts, None, ws, ws_bytes, stream)
+        select(q, k)
         sa.sa_block_sparse_attention(q, k, v, B, H, N, d, idx, counts, L.cap, mask, w.min_active, 0.0, o, ws,
                                      ws_bytes, stream)
         comp_done[i].record(stream)
@@ -356,7 +368,8 @@ def run_ours(args):
     achieved = flops_step / (att_ms * 1e-3) / 1e12
     traffic = traffic_from_profile(os.path.join(ROOT, "prompt_aware_head_b200", "csrc", "attention.cu"))
     n_act = int(mask.sum())
-    sel_bytes = 2.0 * B * n_act * N * d * 2 + 4.0 * tiles + 4.0 * B * n_act * w.nB
+    # a control pattern reads no Q or K: only its lists count
+    sel_bytes = (2.0 * B * n_act * N * d * 2 if args.pattern == "content" else 0.0) + 4.0 * tiles + 4.0 * B * n_act * w.nB
     sel_gbs = sel_bytes / (sel_ms * 1e-3) / 1e9
     out = {
         "metric": METRIC,
@@ -373,7 +386,7 @@ def run_ours(args):
         "data": "synthetic (seeded; Q/K rank-8 sinusoidal position structure + noise, V ~ N(0,1); no weights)",
         "config": {
             "workload": describe(w, rho),
-            "B": B, "H": H, "N": N, "d": d, "density_budget": rho,
+            "B": B, "H": H, "N": N, "d": d, "density_budget": rho, "lists": args.pattern,
             "density_realized": round(tiles / (B * n_act * w.nB ** 2), 5),
             "selected_tiles": int(tiles),
             "l2": "flushed between steps (512 MB write outside the per-step events)" if flush
@@ -459,6 +472,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="joint")
     ap.add_argument("--density", type=float, default=None)
+    ap.add_argument("--pattern", choices=["content", "radial", "window"], default="content",
+                    help="block lists from the content selector (default), or a control pattern at the same pins: "
+                         "radial band at the same k, or a 512-token window + 8 global blocks")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
