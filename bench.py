@@ -54,6 +54,25 @@ def describe(w, rho):
         (", head mask %d of %d" % (int(head_mask_for_layer(w).sum()), w.H)) if w.head_mask or w.mask_runs else "")
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(x, device):
+    """The largest x over all ranks of the process group (x itself with one
+    rank): a step's time is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(flops_per_rank, ms_max, world):
+    """Whole-job effective TFLOP/s: every rank's flops over the slowest rank's
+    time (each rank runs its own batch: weak scaling)."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ oracle (CPU) sample
 def oracle_sample(w, rho, target_s=10.0, seed=0):
     """Times the fp64 oracle on whole heads of the workload (selection for the
@@ -280,12 +299,8 @@ def run_ours(args):
     t_plan = [e[1].elapsed_time(e[2]) for e in evs]
     t_att = [e[2].elapsed_time(e[3]) for e in evs]
     ms_step = statistics.mean(t_step)
-    ms_max = ms_step
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-    value = world * flops_step / (ms_max * 1e-3) / 1e12
+    ms_max = max_over_ranks(ms_step, dev)
+    value = job_value(flops_step, ms_max, world)
     assert sa.sa_check(ws, stream) == sa.SA_OK
 
     # dense baseline (same library, all heads, same inputs), and torch SDPA
@@ -355,12 +370,8 @@ def run_ours(args):
         out_done[i].record(s_out)
     ee[1].record(s_out)
     torch.cuda.synchronize()
-    e2e_ms = ee[0].elapsed_time(ee[1]) / e2e_steps
+    e2e_ms = max_over_ranks(ee[0].elapsed_time(ee[1]) / e2e_steps, dev)
     del slots
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
 
     pk, pk_kind = peaks()
     att_ms = statistics.mean(t_att)
@@ -416,7 +427,7 @@ def run_ours(args):
             "bound": "hbm", "achieved": round(sel_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(sel_gbs / pk["hbm_gbs"], 4), "algorithmic_bytes": int(sel_bytes),
         },
-        "e2e": {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+        "e2e": {"value": round(job_value(flops_step, e2e_ms, world), 3), "unit": UNIT,
                 "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(O.numel() * 2),
                 "ms_per_step": round(e2e_ms, 4),
                 "copies": "pinned host buffers; step i+1's inputs in and step i-1's O out overlap step i"},
