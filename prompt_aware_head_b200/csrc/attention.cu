@@ -373,6 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_dep_wait();  // the work items come from the planner
   const uint32_t tm = *tmem_slot;
   const int G = gridDim.x, cta = blockIdx.x;
   const int total = a.dense ? a.n_items_host : *reinterpret_cast<const volatile int*>(a.n_items_dev);
@@ -747,6 +748,7 @@ __global__ void __launch_bounds__(256) plan_rows_kernel(const int32_t* __restric
                                                         int* __restrict__ err) {
   __shared__ uint32_t bm[8][kWords];
   __shared__ int part[8][3];
+  grid_dep_wait();
   const int bh = blockIdx.y, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * 8 + w, BH = gridDim.y;
   if (!((head_bits >> (bh % H)) & 1ull)) return;
@@ -844,6 +846,8 @@ __global__ void __launch_bounds__(kOrderThreads) plan_order_kernel(const int* __
                                                                    int* __restrict__ n_items) {
   __shared__ uint32_t keys[kMaxBlocks];
   __shared__ int nkeys, best_si, base_sh, total_sh;
+  grid_dep_launch();  // the attention kernel may set up on the SMs this small grid leaves idle
+  grid_dep_wait();
   const int bh = blockIdx.x, t = threadIdx.x;
   if (t == 0) {
     nkeys = 0;
@@ -977,8 +981,7 @@ static cudaError_t launch_attn_kernel(const void* Q, const void* K, const void* 
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << (di.id & 31);
   }
-  sparse_attn_kernel<D><<<di.sm_count, kThreads, AttnSmem<D>::kAlloc, s>>>(mq, mk, mv, args);
-  return cudaGetLastError();
+  return launch_pdl(sparse_attn_kernel<D>, dim3(di.sm_count), dim3(kThreads), AttnSmem<D>::kAlloc, s, mq, mk, mv, args);
 }
 
 static cudaError_t launch_attn(const void* Q, const void* K, const void* V, int BH, int N, int d,
@@ -997,11 +1000,11 @@ cudaError_t launch_attention_plan(const int32_t* idx, const int32_t* counts, int
   int32_t* ulist = reinterpret_cast<int32_t*>(base + wl.ulist);
   int* lens = reinterpret_cast<int*>(base + wl.lens);
   int* partials = reinterpret_cast<int*>(base + wl.totals);
-  plan_rows_kernel<<<dim3(nparts, BH), 256, 0, s>>>(idx, counts, nB, cap, H, head_bits, ulist, lens, partials,
-                                                    &hdr->err);
-  plan_order_kernel<<<BH, kOrderThreads, 0, s>>>(lens, partials, nparts, nB, BH, H, head_bits, items,
-                                                 &hdr->n_items);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(plan_rows_kernel, dim3(nparts, BH), dim3(256), 0, s, idx, counts, nB, cap, H, head_bits,
+                             ulist, lens, partials, &hdr->err);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(plan_order_kernel, dim3(BH), dim3(kOrderThreads), 0, s, static_cast<const int*>(lens),
+                    static_cast<const int*>(partials), nparts, nB, BH, H, head_bits, items, &hdr->n_items);
 }
 
 cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int N, int d,

@@ -45,6 +45,15 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// A kernel launched with programmatic stream serialization (launch_pdl) may
+// start while the previous kernel of its stream is finishing; grid_dep_wait
+// returns once that kernel has completed and its writes are visible (at once
+// when the kernel was launched without the attribute).  grid_dep_launch lets
+// the next kernel start before this one ends.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -21,6 +21,25 @@ struct sa_layout {
 
 namespace sa {
 
+// Launches a kernel that may overlap the end of the previous kernel in its
+// stream (programmatic dependent launch); the kernel calls grid_dep_wait()
+// before it touches anything that kernel wrote.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr{};
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Workspace layout (byte offsets from the caller's workspace base).
 struct WsLayout {
   size_t header = 0;        // WsHeader (256 B)

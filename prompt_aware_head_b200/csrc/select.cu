@@ -331,6 +331,7 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
                                                    const __nv_bfloat16* __restrict__ K, float* __restrict__ qimg,
                                                    float* __restrict__ kimg, int N, int nB, int RT, int H,
                                                    uint64_t head_bits, int bh0, size_t lo_offset) {
+  grid_dep_wait();
   const int i = blockIdx.x, slot = blockIdx.y, bh = bh0 + slot;
   if (!((head_bits >> (bh % H)) & 1ull)) return;
   constexpr int TPR = D / 8;     // threads per row, 8 bf16 (16 B) each
@@ -454,6 +455,7 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(const __grid_constant_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_dep_wait();  // the images come from the previous kernel
   const uint32_t tmem = *tslot;
   bool ok = true;
   if (t == 0) {
@@ -559,6 +561,7 @@ __global__ void __launch_bounds__(128, NC <= 17 ? 8 : 4) rank_rows_kernel(const 
   __shared__ uint32_t memk[4][32];
   __shared__ uint8_t cls[32 * NC];
   __shared__ uint32_t pin_m[NC], sparse_m[NC], drop_m[NC];  // class masks of key blocks 32c + lane
+  grid_dep_wait();
   for (int j = threadIdx.x; j < nB; j += 128) cls[j] = cls_g[j];
   __syncthreads();
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, slot = blockIdx.y, bh = bh0 + slot;
@@ -731,9 +734,8 @@ static cudaError_t ensure_smem(F* kernel, size_t bytes, bool* configured, std::m
 template <int NC>
 static cudaError_t launch_rank_t(const float* scores, const sa_layout* L, int bh0, int nbh, int H, uint64_t head_bits,
                                  int k, int32_t* idx, int32_t* counts, cudaStream_t s) {
-  rank_rows_kernel<NC><<<dim3((L->nB + 7) / 8, nbh), 128, 0, s>>>(scores, L->d_cls, L->nB, H, head_bits, k, L->cap,
-                                                                 idx, counts, bh0);
-  return cudaGetLastError();
+  return launch_pdl(rank_rows_kernel<NC>, dim3((L->nB + 7) / 8, nbh), dim3(128), 0, s, scores,
+                    static_cast<const uint8_t*>(L->d_cls), L->nB, H, head_bits, k, L->cap, idx, counts, bh0);
 }
 
 static cudaError_t launch_rank(int nc, const float* scores, const sa_layout* L, int bh0, int nbh, int H,
@@ -773,16 +775,16 @@ static cudaError_t select_heads(const sa_layout* L, const void* Q, const void* K
   const size_t lo = static_cast<size_t>(nbh) * img_floats(nB, d);
   const auto* q = static_cast<const __nv_bfloat16*>(Q);
   const auto* kk = static_cast<const __nv_bfloat16*>(K);
-  if (d == 128)
-    pool_kernel<128><<<dim3(nB, nbh), 128, 0, s>>>(q, kk, qimg, kimg, L->N, nB, RT, H, head_bits, bh0, lo);
-  else
-    pool_kernel<64><<<dim3(nB, nbh), 128, 0, s>>>(q, kk, qimg, kimg, L->N, nB, RT, H, head_bits, bh0, lo);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = d == 128 ? launch_pdl(pool_kernel<128>, dim3(nB, nbh), dim3(128), 0, s, q, kk, qimg, kimg, L->N, nB, RT, H,
+                            head_bits, bh0, lo)
+               : launch_pdl(pool_kernel<64>, dim3(nB, nbh), dim3(128), 0, s, q, kk, qimg, kimg, L->N, nB, RT, H,
+                            head_bits, bh0, lo);
+  if (e != cudaSuccess) return e;
   TcArgs ta{qimg, kimg, scores, err, lo, nB, RT, H, bh0, head_bits};
   const dim3 grid((nB + kTcN - 1) / kTcN, RT, nbh);
-  if (d == 128) score_tc_kernel<128><<<grid, 128, kTcSmem, s>>>(ta);
-  else score_tc_kernel<64><<<grid, 128, kTcSmem, s>>>(ta);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = d == 128 ? launch_pdl(score_tc_kernel<128>, grid, dim3(128), kTcSmem, s, ta)
+               : launch_pdl(score_tc_kernel<64>, grid, dim3(128), kTcSmem, s, ta);
+  if (e != cudaSuccess) return e;
   return launch_rank(nc, scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
 }
 
