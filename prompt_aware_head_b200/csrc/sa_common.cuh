@@ -16,6 +16,9 @@ constexpr int kMaxHeads = 64;           // head_mask bits
 
 enum BlockClass : uint8_t { kPin = 0, kSparse = 1, kDrop = 2 };
 
+// Attention work items and union lists mark "no second query block" with this.
+constexpr int kNoBlock = 0xFFFF;
+
 // Error bits in the workspace header (mapped to sa_status by the host).
 enum ErrBits : int { kErrBadIndex = 1, kErrTimeout = 2, kErrSmemAlign = 4 };
 
