@@ -140,7 +140,9 @@ SA_API int sa_budget(float density, int n_cand);
  * sa_select_blocks [SDN "selector" + "host sync" paragraphs].
  * Per (batch, active head, 64-row query block i):
  *   qbar_i = mean of the 64 Q rows, kbar_j likewise (fp32 accumulation);
- *   s_ij = qbar_i . kbar_j in fp32, with no scale and no softmax;
+ *   s_ij = qbar_i . kbar_j as an fp32 value, with no scale and no softmax
+ *   (computed on the tensor cores with each mean split into a tf32 part and
+ *   its remainder: each product within about 2^-22 |q||k| of exact);
  *   a SPARSE row keeps its diagonal block, then the k-1 highest-scoring
  *   other SPARSE blocks (ties: lower block index; -0 ranks as +0), plus every
  *   PIN block; k = sa_budget(density, C).  A PIN row keeps every non-DROP
