@@ -1,4 +1,4 @@
-// Host-side internals shared by the C ABI (api.cpp) and the kernel launchers.
+// Host-side internals shared by the C ABI (api.cu) and the kernel launchers.
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -73,7 +73,7 @@ cudaError_t launch_pattern(const sa_layout* L, int kind, int W, int G, int r, in
 cudaError_t launch_density(const int32_t* counts, int B, int H, int nB, uint64_t head_bits, void* ws,
                            unsigned long long* host_tiles, cudaStream_t s);
 
-// Attention launchers (attention.cu).
+// Work plan (plan.cu) and attention launchers (attention.cu).
 cudaError_t launch_attention_plan(const int32_t* idx, const int32_t* counts, int B, int H, int N, int d, int cap,
                                   uint64_t head_bits, void* ws, cudaStream_t s);
 cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
