@@ -7,7 +7,10 @@
 // keep the diagonal.  The "layout" paragraph adds the pins (text / other
 // rows and columns dense) and drops (padding).  The "host sync" paragraph
 // asks for ranking with no host-side k and density read back on demand.
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "sa_common.cuh"
@@ -280,7 +283,8 @@ __device__ __forceinline__ uint32_t warp_topk_bucket(const float (&s)[NC], uint3
 //                      split into a tf32 part and the fp32 remainder, written
 //                      straight into the operand images the tensor cores read;
 //   score_tc_kernel  - one CTA per 128 x 256 tile of a head's scores: bulk
-//                      copies of the images, 3xTF32 MMAs into TMEM;
+//                      copies of the images, 3xTF32 MMAs into TMEM, tensor
+//                      stores of the scores;
 //   rank_rows_kernel - one warp per row keeps the pins, the diagonal and the
 //                      top k - 1 scores (bucket select).
 // Kernel boundaries order the three, so every image is complete before a
@@ -384,6 +388,22 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
   }
 }
 
+// 3D tiled store (no multicast) of a shared-memory box to global memory,
+// tracked by the issuing thread's bulk-async group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until at most n of this thread's bulk stores still read shared memory.
+template <int n>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(n) : "memory");
+}
+
 struct TcArgs {
   const float* qimg;  // q hi images; q lo at + lo_offset
   const float* kimg;  // k hi images; k lo at + lo_offset
@@ -391,6 +411,7 @@ struct TcArgs {
   int* err;
   size_t lo_offset;
   int nB, RT, H, bh0;
+  int tma_store;  // 1: scores leave through the tensor map (3D [slot][nB][nB] fp32, 128-byte swizzle)
   uint64_t head_bits;
 };
 
@@ -423,11 +444,14 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // n0 = 256 blockIdx.x + c (row tiles 2 blockIdx.x and 2 blockIdx.x + 1 of B).
 // Thread 0 streams the d chunks' images through two stages with bulk copies
 // and issues each chunk's MMAs once its stage is full; the MMA commit frees
-// the stage.  Warp w then reads TMEM lanes 32 w .. 32 w + 31 (tile rows) and
-// writes its rows' scores.  Image rows past nB hold whatever was there: they
-// only reach scores that are never written out.
+// the stage.  Warp w then reads TMEM lanes 32 w .. 32 w + 31 (tile rows);
+// the scores leave through tensor stores of 128 x 32 boxes staged in the
+// drained stage buffers, or, where the score rows do not fit a tensor map,
+// as each warp's row stores.  Image rows past nB hold whatever was there:
+// they only reach scores that are never written out.
 template <int D>
-__global__ void __launch_bounds__(128, 1) score_tc_kernel(const __grid_constant__ TcArgs a) {
+__global__ void __launch_bounds__(128, 1) score_tc_kernel(const __grid_constant__ TcArgs a,
+                                                          const __grid_constant__ CUtensorMap ms) {
   constexpr int NKC = D / 32;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -516,7 +540,34 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(const __grid_constant_
   ok = __syncthreads_and(ok ? 1 : 0) != 0;
   if (ok) ok = __syncthreads_and(mbar_wait(done, 0, abort_flag, a.err) ? 1 : 0) != 0;
   tc_fence_after();
-  if (ok) {
+  if (ok && a.tma_store) {
+    // Each 32-column block: TMEM -> registers (lane = tile row) -> a 128 x 32
+    // fp32 box in shared memory, 128-byte swizzled (row r at byte 128 r, its
+    // 16-byte group g at g ^ (r & 7)), two boxes alternating -> one tensor
+    // store per box; the store clips rows and columns past nB.
+    const int r = 32 * w + lane;
+#pragma unroll 1
+    for (int cb = 0; cb < kTcN / 32; ++cb) {
+      const int j0 = n0 + 32 * cb;
+      if (j0 >= nB) break;
+      unsigned char* box = sm + (cb & 1) * kImgBytes;
+      if (cb >= 2) {  // the store issued from this box two blocks ago has read it
+        if (t == 0) bulk_wait_read<1>();
+        __syncthreads();
+      }
+      uint32_t v[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * w) << 16) + 32 * cb, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        *reinterpret_cast<uint4*>(box + r * 128 + ((g ^ (r & 7)) << 4)) =
+            make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic stores -> the store's reads
+      __syncthreads();
+      if (t == 0) tma_store_3d(&ms, box, j0, m0, slot);
+    }
+    if (t == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  } else if (ok) {
     const int i = m0 + 32 * w + lane;
     float* out = a.scores + (static_cast<size_t>(slot) * nB + i) * nB;
 #pragma unroll 1
@@ -753,6 +804,36 @@ static cudaError_t launch_rank(int nc, const float* scores, const sa_layout* L, 
   }
 }
 
+// The driver's tensor-map encoder, looked up once.
+static PFN_cuTensorMapEncodeTiled_v12000 score_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Scores [nbh][nB][nB] fp32 as a 3D tensor (columns, rows, slots), boxes of
+// 32 columns x 128 rows, 128-byte swizzle.  Needs rows of whole 16-byte
+// groups (nB % 4 == 0) and a 16-byte aligned base; false otherwise.
+static bool make_score_map(CUtensorMap* map, float* scores, int nB, int nbh) {
+  if ((nB & 3) != 0 || (reinterpret_cast<uintptr_t>(scores) & 15) != 0) return false;
+  auto enc = score_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(nB), static_cast<cuuint64_t>(nB), static_cast<cuuint64_t>(nbh)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(nB) * 4, static_cast<cuuint64_t>(nB) * nB * 4};
+  cuuint32_t box[3] = {32, kTcM, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, scores, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Floats of one head's image array (hi or lo).
 static size_t img_floats(int nB, int d) { return static_cast<size_t>((nB + kTcM - 1) / kTcM) * d * kTcM; }
 
@@ -780,10 +861,13 @@ static cudaError_t select_heads(const sa_layout* L, const void* Q, const void* K
                : launch_pdl(pool_kernel<64>, dim3(nB, nbh), dim3(128), 0, s, q, kk, qimg, kimg, L->N, nB, RT, H,
                             head_bits, bh0, lo);
   if (e != cudaSuccess) return e;
-  TcArgs ta{qimg, kimg, scores, err, lo, nB, RT, H, bh0, head_bits};
+  CUtensorMap ms;
+  std::memset(&ms, 0, sizeof ms);
+  const int tma_store = make_score_map(&ms, scores, nB, nbh) ? 1 : 0;  // else plain row stores
+  TcArgs ta{qimg, kimg, scores, err, lo, nB, RT, H, bh0, tma_store, head_bits};
   const dim3 grid((nB + kTcN - 1) / kTcN, RT, nbh);
-  e = d == 128 ? launch_pdl(score_tc_kernel<128>, grid, dim3(128), kTcSmem, s, ta)
-               : launch_pdl(score_tc_kernel<64>, grid, dim3(128), kTcSmem, s, ta);
+  e = d == 128 ? launch_pdl(score_tc_kernel<128>, grid, dim3(128), kTcSmem, s, ta, ms)
+               : launch_pdl(score_tc_kernel<64>, grid, dim3(128), kTcSmem, s, ta, ms);
   if (e != cudaSuccess) return e;
   return launch_rank(nc, scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
 }

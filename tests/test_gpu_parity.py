@@ -91,6 +91,22 @@ def test_select_parity(sa, name, rho):
         print("%s rho=%.1f: %d rows rank differently under fp64 scores" % (name, rho, diff))
 
 
+@pytest.mark.parametrize("nB", [131, 132, 262])
+def test_select_parity_ragged_block_count(sa, nB):
+    # a multiple of 4 blocks: scores leave in 128 x 32 tensor-store boxes clipped at nB; otherwise as row stores
+    N = 64 * nB
+    w = make_workload("tiny", N=N, d=128, H=2, head_mask=None, min_active=0,
+                      segments=((SEG_TEXT, 0, 64), (SEG_PAD, 64, 64), (SEG_IMAGE, 128, N - 128)))
+    Q, K, _ = make_qkv(w, seed=nB)
+    L, buf, sc = _select(sa, w, Q, K, 0.3, None, 0)
+    _check_scores(w, Q, K, sc, None)
+    cls = oracle.layout(list(w.segments), w.N)
+    ref_idx, ref_cnt = oracle.select(sc.reshape(-1, w.nB, w.nB).astype(np.float64), cls, w.H, 0.3,
+                                     np.ones(w.H, np.uint8), cap=L.cap)
+    idx, cnt = buf.lists()
+    compare_lists(idx, cnt, ref_idx, ref_cnt)
+
+
 @pytest.mark.parametrize("layer", [0, 1, 63])
 @pytest.mark.parametrize("rho", [1.0, 0.5])
 def test_select_parity_stack(sa, layer, rho):
