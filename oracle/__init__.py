@@ -45,13 +45,13 @@ def _load():
         _lib.oracle_layout.argtypes = [P, i, i, i, P]
         _lib.oracle_layout.restype = i
         _lib.oracle_pool.argtypes = [P, i, i, i, i, P]
-        _lib.oracle_scores.argtypes = [P, P, i, i, i, P]
+        _lib.oracle_scores.argtypes = [P, P, i, i, i, i, i, P]
         _lib.oracle_budget.argtypes = [f, i]
         _lib.oracle_budget.restype = i
         _lib.oracle_select.argtypes = [P, P, i, i, i, f, P, i, P, P]
         _lib.oracle_pattern.argtypes = [P, i, i, i, i, i, i, f, i, i, P, i, P, P]
         _lib.oracle_pattern.restype = i
-        _lib.oracle_attention.argtypes = [P, P, P, i, i, i, i, i, P, P, i, P, dbl, P, ctypes.c_int64, P]
+        _lib.oracle_attention.argtypes = [P, P, P, i, i, i, i, i, i, P, P, i, P, dbl, P, ctypes.c_int64, P]
         _lib.oracle_density.argtypes = [P, i, i, i, P, P, P]
     return _lib
 
@@ -82,15 +82,31 @@ def pool(X: np.ndarray, block: int = 64) -> np.ndarray:
     return out.reshape(X.shape[:-2] + (N // block, d))
 
 
+def _kv_heads(H: int, q_size: int, k_size: int) -> int:
+    """Key/value heads when a query tensor of q_size elements has H heads and
+    the key tensor k_size elements (same batch, length and head size)."""
+    if k_size * H % q_size != 0:
+        raise ValueError("key tensor does not hold a whole number of heads")
+    Hkv = k_size * H // q_size
+    if Hkv < 1 or H % Hkv != 0:
+        raise ValueError("query heads %d are not a multiple of key/value heads %d" % (H, Hkv))
+    return Hkv
+
+
 def scores(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
-    """s[i][j] = qbar_i . kbar_j in fp64 (no scale, no softmax)."""
+    """s[i][j] = qbar_i . kbar_j in fp64 (no scale, no softmax), on query heads.
+
+    qbar [..., H, nB, d]; kbar [..., Hkv, nB, d] with H a multiple of Hkv
+    (grouped heads: query head h scores against key head h // (H / Hkv))."""
     lib = _load()
     qbar = np.ascontiguousarray(qbar, dtype=np.float64)
     kbar = np.ascontiguousarray(kbar, dtype=np.float64)
     nB, d = qbar.shape[-2], qbar.shape[-1]
     BH = int(np.prod(qbar.shape[:-2])) if qbar.ndim > 2 else 1
+    H = qbar.shape[-3] if qbar.ndim > 2 else 1
+    Hkv = _kv_heads(H, qbar.size, kbar.size)
     out = np.zeros((BH, nB, nB), dtype=np.float64)
-    lib.oracle_scores(_ptr(qbar), _ptr(kbar), BH, nB, d, _ptr(out))
+    lib.oracle_scores(_ptr(qbar), _ptr(kbar), BH, H, Hkv, nB, d, _ptr(out))
     return out.reshape(qbar.shape[:-2] + (nB, nB))
 
 
@@ -140,7 +156,9 @@ def pattern(cls: np.ndarray, kind: int, BH: int, H: int, window: int = 0, n_glob
 def attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, H: int, idx: np.ndarray, counts: np.ndarray,
               head_mask: Optional[np.ndarray] = None, scale: Optional[float] = None,
               rows: Optional[np.ndarray] = None, block: int = 64) -> np.ndarray:
-    """fp64 attention over the kept tiles; Q/K/V uint16 bf16 bits [B, H, N, d].
+    """fp64 attention over the kept tiles; Q uint16 bf16 bits [B, H, N, d],
+    K and V [B, Hkv, N, d] with H a multiple of Hkv (query head h reads
+    key/value head h // (H / Hkv)).
 
     rows: flat row ids (b*H + h)*N + n to compute (None = all); returns
     [len(rows), d] (or [B, H, N, d] when rows is None)."""
@@ -150,6 +168,9 @@ def attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, H: int, idx: np.ndarr
     V = np.ascontiguousarray(V, dtype=np.uint16)
     N, d = Q.shape[-2], Q.shape[-1]
     BH = int(np.prod(Q.shape[:-2]))
+    Hkv = _kv_heads(H, Q.size, K.size)
+    if V.size != K.size:
+        raise ValueError("K and V differ in size")
     idx = np.ascontiguousarray(idx, dtype=np.int32)
     counts = np.ascontiguousarray(counts, dtype=np.int32)
     cap = idx.shape[-1]
@@ -157,12 +178,12 @@ def attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, H: int, idx: np.ndarr
     sc = 1.0 / np.sqrt(d) if scale is None else float(scale)
     if rows is None:
         out = np.zeros((BH * N, d), dtype=np.float64)
-        lib.oracle_attention(_ptr(Q), _ptr(K), _ptr(V), BH, H, N, d, block, _ptr(idx), _ptr(counts), cap,
+        lib.oracle_attention(_ptr(Q), _ptr(K), _ptr(V), BH, H, Hkv, N, d, block, _ptr(idx), _ptr(counts), cap,
                              _ptr(hm), sc, None, BH * N, _ptr(out))
         return out.reshape(Q.shape)
     rows = np.ascontiguousarray(rows, dtype=np.int64)
     out = np.zeros((rows.shape[0], d), dtype=np.float64)
-    lib.oracle_attention(_ptr(Q), _ptr(K), _ptr(V), BH, H, N, d, block, _ptr(idx), _ptr(counts), cap,
+    lib.oracle_attention(_ptr(Q), _ptr(K), _ptr(V), BH, H, Hkv, N, d, block, _ptr(idx), _ptr(counts), cap,
                          _ptr(hm), sc, _ptr(rows), rows.shape[0], _ptr(out))
     return out
 

@@ -107,19 +107,30 @@ void oracle_pool(const uint16_t* X, int BH, int N, int d, int block, double* out
 }
 
 /*
- * Tile-pair scores s[i][j] = qbar_i . kbar_j, no scale and no softmax
- * [SDN "selector": top-k is invariant under both].  [BH][nB][nB] fp64.
+ * The key/value head that query head bh = b*H + h reads when H query heads
+ * share Hkv key/value heads [SDN "selector": scoring runs on query heads, so
+ * grouped attention needs no key expansion]: consecutive groups of H/Hkv
+ * query heads share one, b*Hkv + h / (H/Hkv).  Hkv = H is plain multi-head.
  */
-void oracle_scores(const double* qbar, const double* kbar, int BH, int nB, int d, double* s) {
+static int kv_head(int bh, int H, int Hkv) { return (bh / H) * Hkv + (bh % H) / (H / Hkv); }
+
+/*
+ * Tile-pair scores s[i][j] = qbar_i . kbar_j, no scale and no softmax
+ * [SDN "selector": top-k is invariant under both], on query heads: qbar is
+ * [BH][nB][d] (BH = B*H), kbar [B*Hkv][nB][d], s [BH][nB][nB] fp64.
+ */
+void oracle_scores(const double* qbar, const double* kbar, int BH, int H, int Hkv, int nB, int d, double* s) {
 #pragma omp parallel for schedule(static)
-  for (int bh = 0; bh < BH; ++bh)
+  for (int bh = 0; bh < BH; ++bh) {
+    int kh = kv_head(bh, H, Hkv);
     for (int i = 0; i < nB; ++i)
       for (int j = 0; j < nB; ++j) {
         double acc = 0.0;
         for (int c = 0; c < d; ++c)
-          acc += qbar[((size_t)bh * nB + i) * d + c] * kbar[((size_t)bh * nB + j) * d + c];
+          acc += qbar[((size_t)bh * nB + i) * d + c] * kbar[((size_t)kh * nB + j) * d + c];
         s[((size_t)bh * nB + i) * nB + j] = acc;
       }
+  }
 }
 
 /* Budget in candidates [SDN "selector": a fraction of the sparsifiable candidates]. */
@@ -286,11 +297,12 @@ int oracle_pattern(const uint8_t* cls, int nB, int block, int kind, int W, int G
  * Attention over the selected tiles [GLO block-sparse; SDN flex consumer:
  * every selected tile computed in full].  For each requested query row:
  * S = q . K^T * scale, -inf outside the kept tiles, softmax, times V.
- * Rows whose list is empty, and skipped heads, give O = 0.  Q, K, V are
- * bf16 bits [BH][N][d]; rows lists flat row ids bh*N + n (NULL = every
- * row); out is [nrows][d] fp64.
+ * Rows whose list is empty, and skipped heads, give O = 0.  Q is bf16 bits
+ * [BH][N][d]; K and V are [B*Hkv][N][d], query head bh reading key/value
+ * head kv_head(bh); rows lists flat row ids bh*N + n (NULL = every row);
+ * out is [nrows][d] fp64.
  */
-void oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int BH, int H, int N, int d,
+void oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int BH, int H, int Hkv, int N, int d,
                       int block, const int32_t* idx, const int32_t* counts, int cap, const uint8_t* head_mask,
                       double scale, const int64_t* rows, int64_t nrows, double* out) {
   int nB = N / block;
@@ -303,7 +315,7 @@ void oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
 #pragma omp for schedule(dynamic, 16)
     for (int64_t t = 0; t < nrows; ++t) {
       int64_t row = rows ? rows[t] : t;
-      int bh = (int)(row / N), n = (int)(row % N), i = n / block;
+      int bh = (int)(row / N), n = (int)(row % N), i = n / block, kh = kv_head(bh, H, Hkv);
       double* o = out + (size_t)t * d;
       for (int c = 0; c < d; ++c) o[c] = 0.0;
       int active = head_mask ? head_mask[bh % H] != 0 : 1;
@@ -318,7 +330,7 @@ void oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
       for (int key = 0; key < N; ++key) {
         if (!keep[key]) { s[key] = -INFINITY; continue; }
         double acc = 0.0;
-        for (int c = 0; c < d; ++c) acc += q[c] * bf16_to_double(K[((size_t)bh * N + key) * d + c]);
+        for (int c = 0; c < d; ++c) acc += q[c] * bf16_to_double(K[((size_t)kh * N + key) * d + c]);
         s[key] = acc * scale;
         if (s[key] > mx) mx = s[key];
       }
@@ -327,7 +339,7 @@ void oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
         if (!keep[key]) continue;
         double p = exp(s[key] - mx);
         den += p;
-        for (int c = 0; c < d; ++c) o[c] += p * bf16_to_double(V[((size_t)bh * N + key) * d + c]);
+        for (int c = 0; c < d; ++c) o[c] += p * bf16_to_double(V[((size_t)kh * N + key) * d + c]);
       }
       for (int c = 0; c < d; ++c) o[c] /= den;
     }

@@ -357,3 +357,42 @@ def test_attention_rows_subset_matches_full():
     full = oracle.attention(Q, K, V, w.H, idx, counts).reshape(-1, w.d)
     rows = np.array([0, 77, 130, 511, 512 + 200, 3 * 512 + 511])
     np.testing.assert_array_equal(oracle.attention(Q, K, V, w.H, idx, counts, rows=rows), full[rows])
+
+
+# ---------------------------------------------------------------- grouped key/value heads
+
+def test_grouped_attention_dense_equals_sdpa_gqa():
+    # 6 query heads over 2 key/value heads, two batches: torch SDPA's grouped mode in fp64
+    rng = np.random.default_rng(8)
+    Q = _bits(rng.standard_normal((2, 6, 256, 64)))
+    K, V = (_bits(rng.standard_normal((2, 2, 256, 64))) for _ in range(2))
+    cls = oracle.layout([], 256)
+    idx, counts = oracle.select(np.zeros((12, 4, 4)), cls, 6, 1.0)
+    got = oracle.attention(Q, K, V, 6, idx, counts)
+    ref = torch.nn.functional.scaled_dot_product_attention(*(torch.from_numpy(_f64(x)) for x in (Q, K, V)),
+                                                           enable_gqa=True).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_heads_equal_multi_head_on_repeated_keys():
+    # sharing a key/value head is multi-head attention on keys and values repeated per group
+    w = WORKLOADS["tiny"]
+    rng = np.random.default_rng(9)
+    B, H, Hkv, N, d = 2, 4, 2, w.N, 64
+    Q = _bits(rng.standard_normal((B, H, N, d)))
+    K, V = (_bits(rng.standard_normal((B, Hkv, N, d))) for _ in range(2))
+    Kr, Vr = (np.repeat(x, H // Hkv, axis=1) for x in (K, V))
+    qbar, kbar = oracle.pool(Q), oracle.pool(K)
+    s = oracle.scores(qbar, kbar)
+    np.testing.assert_array_equal(s, oracle.scores(qbar, oracle.pool(Kr)))
+    assert not np.array_equal(s[0, 1], s[0, 2])  # heads 1 and 2 read different key heads
+    cls = oracle.layout(list(w.segments), N)
+    idx, counts = oracle.select(s.reshape(-1, w.nB, w.nB), cls, H, 0.5)
+    np.testing.assert_array_equal(oracle.attention(Q, K, V, H, idx, counts),
+                                  oracle.attention(Q, Kr, Vr, H, idx, counts))
+
+
+def test_grouped_heads_reject_a_partial_group():
+    q = np.zeros((1, 6, 2, 8))
+    with pytest.raises(ValueError):
+        oracle.scores(q, np.zeros((1, 4, 2, 8)))
