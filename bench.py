@@ -8,6 +8,7 @@ tiles.  Metric: effective TFLOP/s = 4 * 64 * 64 * d * (selected tiles) / step
 time, i.e. 4*B*H_active*N^2*d*density / t.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload joint|sdxl|video|stack|tiny]
+                  [--pattern content|radial|window] [--kv-heads H_kv]
   python bench.py --impl reference ...     # the fp64 CPU oracle on a bounded sample
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own
@@ -47,11 +48,18 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def describe(w, rho):
+def describe(w, rho, H_kv=None):
     segs = ", ".join("%s[%d,%d)" % ({0: "text", 1: "pad", 2: "image", 3: "other"}[k], s, s + l) for k, s, l in w.segments)
-    return "%s: B%d H%d d%d N%d%s, density %.2f%s" % (
-        w.name, w.B, w.H, w.d, w.N, (" (" + segs + ")") if segs else "", rho,
+    return "%s: B%d H%d%s d%d N%d%s, density %.2f%s" % (
+        w.name, w.B, w.H, (" (K/V heads %d)" % H_kv) if H_kv and H_kv != w.H else "", w.d, w.N,
+        (" (" + segs + ")") if segs else "", rho,
         (", head mask %d of %d" % (int(head_mask_for_layer(w).sum()), w.H)) if w.head_mask or w.mask_runs else "")
+
+
+def grouped_kv(K, V, g):
+    """K and V of the first head of each group of g query heads: the shared
+    key/value heads of a grouped-query layout ([B, H / g, N, d])."""
+    return np.ascontiguousarray(K[:, ::g]), np.ascontiguousarray(V[:, ::g])
 
 
 # ------------------------------------------------------------------ ranks
@@ -74,10 +82,11 @@ def job_value(flops_per_rank, ms_max, world):
 
 
 # ------------------------------------------------------------------ oracle (CPU) sample
-def oracle_sample(w, rho, target_s=10.0, seed=0):
+def oracle_sample(w, rho, target_s=10.0, seed=0, g=1):
     """Times the fp64 oracle on whole heads of the workload (selection for the
     head, then attention for all its query rows) until about target_s of CPU
-    work; very long heads are cut to an evenly spaced subset of rows."""
+    work; very long heads are cut to an evenly spaced subset of rows.  g > 1:
+    each query head reads the key/value head of its group of g."""
     import oracle
     mask = head_mask_for_layer(w)
     heads = [int(h) for h in np.flatnonzero(mask)]
@@ -87,6 +96,8 @@ def oracle_sample(w, rho, target_s=10.0, seed=0):
     done_heads, done_rows = 0, 0
     for h in heads:
         Q, K, V = make_qkv(w, seed=seed, heads=[h])
+        if g > 1:
+            _, K, V = make_qkv(w, seed=seed, heads=[g * (h // g)])
         Q, K, V = Q[:1], K[:1], V[:1]
         t0 = time.perf_counter()
         sc = oracle.scores(oracle.pool(Q), oracle.pool(K)).reshape(-1, w.nB, w.nB)
@@ -221,8 +232,14 @@ def run_ours(args):
     w = WORKLOADS[args.workload]
     rho = args.density if args.density else w.densities[0]
     B, H, N, d = w.B, w.H, w.N, w.d
+    H_kv = args.kv_heads or H
+    if H_kv < 1 or H % H_kv:
+        raise SystemExit("--kv-heads must divide the workload's %d heads" % H)
+    g = H // H_kv
     mask = head_mask_for_layer(w)
     Qh, Kh, Vh = make_qkv(w, seed=rank)
+    if g > 1:
+        Kh, Vh = grouped_kv(Kh, Vh, g)
     pin = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (Qh, Kh, Vh)]
     Q, K, V = (p.to(dev, non_blocking=False) for p in pin)
     L = sa.Layout(list(w.segments), N)
@@ -234,7 +251,7 @@ def run_ours(args):
     O_host = torch.empty(O.shape, dtype=torch.bfloat16).pin_memory()
     stream = torch.cuda.current_stream(dev)
     sa.sa_workspace_init(ws, ws_bytes, stream)
-    in_bytes = 3 * Q.numel() * 2
+    in_bytes = (Q.numel() + K.numel() + V.numel()) * 2
     flush = in_bytes < 2 * L2_BYTES
     scratch = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev) if flush else None
     k_budget = sa.sa_budget(rho, L.n_cand)
@@ -243,7 +260,8 @@ def run_ours(args):
 
     def select(q, k):
         if args.pattern == "content":
-            sa.sa_select_blocks(L, q, k, B, H, d, rho, mask, w.min_active, idx, counts, None, ws, ws_bytes, stream)
+            sa.sa_select_blocks_gqa(L, q, k, B, H, H_kv, d, rho, mask, w.min_active, idx, counts, None, ws, ws_bytes,
+                                    stream)
         elif args.pattern == "radial":
             sa.sa_pattern_mask(L, sa.SA_PAT_RADIAL, B, H, rho, mask, w.min_active, idx, counts, stream=stream)
         else:
@@ -259,7 +277,7 @@ def run_ours(args):
         sa.sa_attention_plan(idx, counts, B, H, N, d, L.cap, mask, w.min_active, ws, ws_bytes, stream)
         if ev is not None:
             ev[2].record(stream)
-        sa.sa_attention_run(Q, K, V, B, H, N, d, mask, w.min_active, 0.0, O, ws, ws_bytes, stream)
+        sa.sa_attention_run_gqa(Q, K, V, B, H, H_kv, N, d, mask, w.min_active, 0.0, O, ws, ws_bytes, stream)
         if ev is not None:
             ev[3].record(stream)
 
@@ -308,18 +326,19 @@ def run_ours(args):
     if not args.no_dense:
         Od = torch.empty_like(O)
         for _ in range(3):
-            sa.sa_dense_attention(Q, K, V, B, H, N, d, 0.0, Od, ws, ws_bytes, stream)
+            sa.sa_dense_attention_gqa(Q, K, V, B, H, H_kv, N, d, 0.0, Od, ws, ws_bytes, stream)
         de = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
         for a, b in de:
             if flush:
                 scratch.fill_(1.0)
             a.record(stream)
-            sa.sa_dense_attention(Q, K, V, B, H, N, d, 0.0, Od, ws, ws_bytes, stream)
+            sa.sa_dense_attention_gqa(Q, K, V, B, H, H_kv, N, d, 0.0, Od, ws, ws_bytes, stream)
             b.record(stream)
         torch.cuda.synchronize()
         dense_ms = statistics.mean(a.elapsed_time(b) for a, b in de)
         try:
-            f = torch.nn.functional.scaled_dot_product_attention
+            def f(q, k, v):
+                return torch.nn.functional.scaled_dot_product_attention(q, k, v, enable_gqa=g > 1)
             for _ in range(2):
                 f(Q, K, V)
             se = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(3)]
@@ -361,8 +380,8 @@ def run_ours(args):
         if i >= 2:
             stream.wait_event(out_done[i - 2])
         select(q, k)
-        sa.sa_block_sparse_attention(q, k, v, B, H, N, d, idx, counts, L.cap, mask, w.min_active, 0.0, o, ws,
-                                     ws_bytes, stream)
+        sa.sa_block_sparse_attention_gqa(q, k, v, B, H, H_kv, N, d, idx, counts, L.cap, mask, w.min_active, 0.0, o,
+                                         ws, ws_bytes, stream)
         comp_done[i].record(stream)
         s_out.wait_event(comp_done[i])
         with torch.cuda.stream(s_out):
@@ -379,8 +398,10 @@ def run_ours(args):
     achieved = flops_step / (att_ms * 1e-3) / 1e12
     traffic = traffic_from_profile(os.path.join(ROOT, "prompt_aware_head_b200", "csrc", "attention.cu"))
     n_act = int(mask.sum())
+    n_kv_act = len({h // g for h in np.flatnonzero(mask)})  # key heads some active query head reads
     # a control pattern reads no Q or K: only its lists count
-    sel_bytes = (2.0 * B * n_act * N * d * 2 if args.pattern == "content" else 0.0) + 4.0 * tiles + 4.0 * B * n_act * w.nB
+    sel_bytes = ((1.0 * B * (n_act + n_kv_act) * N * d * 2 if args.pattern == "content" else 0.0)
+                 + 4.0 * tiles + 4.0 * B * n_act * w.nB)
     sel_gbs = sel_bytes / (sel_ms * 1e-3) / 1e9
     out = {
         "metric": METRIC,
@@ -396,8 +417,8 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic (seeded; Q/K rank-8 sinusoidal position structure + noise, V ~ N(0,1); no weights)",
         "config": {
-            "workload": describe(w, rho),
-            "B": B, "H": H, "N": N, "d": d, "density_budget": rho, "lists": args.pattern,
+            "workload": describe(w, rho, H_kv),
+            "B": B, "H": H, "H_kv": H_kv, "N": N, "d": d, "density_budget": rho, "lists": args.pattern,
             "density_realized": round(tiles / (B * n_act * w.nB ** 2), 5),
             "selected_tiles": int(tiles),
             "l2": "flushed between steps (512 MB write outside the per-step events)" if flush
@@ -435,7 +456,7 @@ def run_ours(args):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = oracle_sample(w, rho, target_s=args.cpu_seconds, seed=rank)
+        cb = oracle_sample(w, rho, target_s=args.cpu_seconds, seed=rank, g=g)
         cb.pop("seconds", None)
         out["cpu_baseline"] = cb
     if world > 1:
@@ -453,12 +474,16 @@ def run_reference(args):
         return
     w = WORKLOADS[args.workload]
     rho = args.density if args.density else w.densities[0]
+    H_kv = args.kv_heads or w.H
+    if H_kv < 1 or w.H % H_kv:
+        raise SystemExit("--kv-heads must divide the workload's %d heads" % w.H)
+    g = w.H // H_kv
     per_step = max(2.0, 120.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        oracle_sample(w, rho, target_s=min(per_step, 2.0))
+        oracle_sample(w, rho, target_s=min(per_step, 2.0), g=g)
     vals, secs, last = [], [], None
     for _ in range(args.steps):
-        last = oracle_sample(w, rho, target_s=per_step)
+        last = oracle_sample(w, rho, target_s=per_step, g=g)
         vals.append(last["value"])
         secs.append(last["seconds"])
     value = statistics.mean(vals)
@@ -467,7 +492,8 @@ def run_reference(args):
         "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(secs), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded generator)",
-        "config": {"workload": describe(w, rho), "B": w.B, "H": w.H, "N": w.N, "d": w.d, "density_budget": rho},
+        "config": {"workload": describe(w, rho, H_kv), "B": w.B, "H": w.H, "H_kv": H_kv, "N": w.N, "d": w.d,
+                   "density_budget": rho},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last["cores"], "kind": "oracle",
                          "sample": last["sample"]},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -486,6 +512,9 @@ def main():
     ap.add_argument("--pattern", choices=["content", "radial", "window"], default="content",
                     help="block lists from the content selector (default), or a control pattern at the same pins: "
                          "radial band at the same k, or a 512-token window + 8 global blocks")
+    ap.add_argument("--kv-heads", type=int, default=None,
+                    help="grouped-query layout: K and V hold this many heads, each shared by H / kv-heads "
+                         "consecutive query heads (default: as many as Q)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -242,6 +242,38 @@ SA_API sa_status sa_dense_attention(const void* Q, const void* K, const void* V,
                              float softmax_scale, void* O, void* ws, size_t ws_bytes, sa_stream_t stream);
 
 /*
+ * Grouped key/value heads [SDN "selector": scoring runs on query heads, so
+ * grouped attention needs no key expansion].  The _gqa forms take K (and V)
+ * with H_kv heads, [B][H_kv][N][d], H a multiple of H_kv: query head h reads
+ * key/value head h / (H / H_kv), so each run of H / H_kv consecutive query
+ * heads shares one.  Selection pools each needed key head once and scores
+ * every query head against its key head's block means; nothing is copied
+ * or expanded.  Q, O, idx, counts, scores_out, the head mask and the
+ * workspace keep their H-head shapes and sizes (sa_workspace_size(B, H, N,
+ * d) covers both forms).  H_kv == H is exactly the plain form (which calls
+ * these); H_kv < 1, H_kv > H or H % H_kv != 0 returns SA_ERR_SHAPE before
+ * any launch.  Everything else is as in the plain form of each call.
+ */
+SA_API sa_status sa_select_blocks_gqa(const sa_layout* L, const void* Q, const void* K, int B, int H, int H_kv,
+                                      int d, float density, const uint8_t* head_mask, int min_active,
+                                      int32_t* idx, int32_t* counts, float* scores_out,
+                                      void* ws, size_t ws_bytes, sa_stream_t stream);
+SA_API sa_status sa_select_blocks_noalloc_gqa(const sa_layout* L, const void* Q, const void* K, int B, int H,
+                                              int H_kv, int d, float density, const uint8_t* head_mask,
+                                              int min_active, int32_t* idx, int32_t* counts, float* scores_out,
+                                              sa_stream_t stream);
+SA_API sa_status sa_block_sparse_attention_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv,
+                                               int N, int d, const int32_t* idx, const int32_t* counts, int cap,
+                                               const uint8_t* head_mask, int min_active, float softmax_scale,
+                                               void* O, void* ws, size_t ws_bytes, sa_stream_t stream);
+SA_API sa_status sa_attention_run_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N,
+                                      int d, const uint8_t* head_mask, int min_active, float softmax_scale, void* O,
+                                      void* ws, size_t ws_bytes, sa_stream_t stream);
+SA_API sa_status sa_dense_attention_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N,
+                                        int d, float softmax_scale, void* O, void* ws, size_t ws_bytes,
+                                        sa_stream_t stream);
+
+/*
  * sa_density [SDN "host sync": density is read back only when something
  * asks].  The only call that reads device memory back: it synchronises
  * `stream`.  Any of the outputs may be NULL.

@@ -68,6 +68,11 @@ _SIGS = {
     "sa_attention_plan": ([_P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _SZ, _P], _I),
     "sa_attention_run": ([_P, _P, _P, _I, _I, _I, _I, _P, _I, _F, _P, _P, _SZ, _P], _I),
     "sa_dense_attention": ([_P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _SZ, _P], _I),
+    "sa_select_blocks_gqa": ([_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P, _P, _SZ, _P], _I),
+    "sa_select_blocks_noalloc_gqa": ([_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P, _P], _I),
+    "sa_block_sparse_attention_gqa": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _F, _P, _P, _SZ, _P], _I),
+    "sa_attention_run_gqa": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _F, _P, _P, _SZ, _P], _I),
+    "sa_dense_attention_gqa": ([_P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _SZ, _P], _I),
     "sa_density": ([_P, _I, _I, _I, _P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
                     ctypes.POINTER(sa_stats), _P, _SZ, _P], _I),
     "sa_workspace_size": ([_I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
@@ -229,6 +234,49 @@ def sa_dense_attention(Q, K, V, B: int, H: int, N: int, d: int, softmax_scale: f
                        stream=None) -> None:
     _check(_lib.sa_dense_attention(_addr(Q), _addr(K), _addr(V), B, H, N, d, ctypes.c_float(softmax_scale),
                                    _addr(O), _addr(ws), ws_bytes, _stream(stream)), "sa_dense_attention")
+
+
+# Grouped key/value heads: K and V hold H_kv heads, query head h reads h // (H // H_kv).
+
+def sa_select_blocks_gqa(L: Layout, Q, K, B: int, H: int, H_kv: int, d: int, density: float, head_mask,
+                         min_active: int, idx, counts, scores_out, ws, ws_bytes: int, stream=None) -> None:
+    mptr, _keep = _host_mask(head_mask)
+    _check(_lib.sa_select_blocks_gqa(L.handle, _addr(Q), _addr(K), B, H, H_kv, d, ctypes.c_float(density), mptr,
+                                     min_active, _addr(idx), _addr(counts), _addr(scores_out), _addr(ws), ws_bytes,
+                                     _stream(stream)), "sa_select_blocks_gqa")
+
+
+def sa_select_blocks_noalloc_gqa(L: Layout, Q, K, B: int, H: int, H_kv: int, d: int, density: float, head_mask,
+                                 min_active: int, idx, counts, scores_out, stream=None) -> None:
+    mptr, _keep = _host_mask(head_mask)
+    _check(_lib.sa_select_blocks_noalloc_gqa(L.handle, _addr(Q), _addr(K), B, H, H_kv, d, ctypes.c_float(density),
+                                             mptr, min_active, _addr(idx), _addr(counts), _addr(scores_out),
+                                             _stream(stream)), "sa_select_blocks_noalloc_gqa")
+
+
+def sa_block_sparse_attention_gqa(Q, K, V, B: int, H: int, H_kv: int, N: int, d: int, idx, counts, cap: int,
+                                  head_mask, min_active: int, softmax_scale: float, O, ws, ws_bytes: int,
+                                  stream=None) -> None:
+    mptr, _keep = _host_mask(head_mask)
+    _check(_lib.sa_block_sparse_attention_gqa(_addr(Q), _addr(K), _addr(V), B, H, H_kv, N, d, _addr(idx),
+                                              _addr(counts), cap, mptr, min_active, ctypes.c_float(softmax_scale),
+                                              _addr(O), _addr(ws), ws_bytes, _stream(stream)),
+           "sa_block_sparse_attention_gqa")
+
+
+def sa_attention_run_gqa(Q, K, V, B: int, H: int, H_kv: int, N: int, d: int, head_mask, min_active: int,
+                         softmax_scale: float, O, ws, ws_bytes: int, stream=None) -> None:
+    mptr, _keep = _host_mask(head_mask)
+    _check(_lib.sa_attention_run_gqa(_addr(Q), _addr(K), _addr(V), B, H, H_kv, N, d, mptr, min_active,
+                                     ctypes.c_float(softmax_scale), _addr(O), _addr(ws), ws_bytes, _stream(stream)),
+           "sa_attention_run_gqa")
+
+
+def sa_dense_attention_gqa(Q, K, V, B: int, H: int, H_kv: int, N: int, d: int, softmax_scale: float, O, ws,
+                           ws_bytes: int, stream=None) -> None:
+    _check(_lib.sa_dense_attention_gqa(_addr(Q), _addr(K), _addr(V), B, H, H_kv, N, d,
+                                       ctypes.c_float(softmax_scale), _addr(O), _addr(ws), ws_bytes,
+                                       _stream(stream)), "sa_dense_attention_gqa")
 
 
 def sa_density(counts, B: int, H: int, nB: int, head_mask, ws, ws_bytes: int, stream=None):

@@ -264,12 +264,15 @@ sa_status sa_check(void* ws, sa_stream_t stream) {
   return SA_OK;
 }
 
-sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, float density,
-                           const uint8_t* head_mask, int min_active, int32_t* idx, int32_t* counts,
-                           float* scores_out, void* ws, size_t ws_bytes, sa_stream_t stream) {
+// Key/value heads: at least one, and H a whole number of groups of them.
+static bool kv_heads_ok(int H, int H_kv) { return H_kv >= 1 && H_kv <= H && H % H_kv == 0; }
+
+sa_status sa_select_blocks_gqa(const sa_layout* L, const void* Q, const void* K, int B, int H, int H_kv, int d,
+                               float density, const uint8_t* head_mask, int min_active, int32_t* idx,
+                               int32_t* counts, float* scores_out, void* ws, size_t ws_bytes, sa_stream_t stream) {
   if (!L || !Q || !K || !idx || !counts) return SA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K)) return SA_ERR_INVALID_ARG;
-  if (B <= 0 || (d != 64 && d != 128)) return SA_ERR_SHAPE;
+  if (B <= 0 || (d != 64 && d != 128) || !kv_heads_ok(H, H_kv)) return SA_ERR_SHAPE;
   if (static_cast<long long>(B) * H * L->N >= (1ll << 31)) return SA_ERR_SHAPE;
   if (!density_ok(density)) return SA_ERR_INVALID_ARG;
   uint64_t bits = 0;
@@ -280,16 +283,23 @@ sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void* K, int
   if ((st = check_device(&di)) != SA_OK) return st;
   if (di.id != L->device) return SA_ERR_INVALID_ARG;
   const int k = sa_budget(density, L->n_cand);
-  return from_cuda(launch_select(L, Q, K, B, H, d, k, bits, idx, counts, scores_out, ws,
+  return from_cuda(launch_select(L, Q, K, B, H, H_kv, d, k, bits, idx, counts, scores_out, ws,
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
-sa_status sa_select_blocks_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int d,
-                                   float density, const uint8_t* head_mask, int min_active, int32_t* idx,
-                                   int32_t* counts, float* scores_out, sa_stream_t stream) {
+sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, float density,
+                           const uint8_t* head_mask, int min_active, int32_t* idx, int32_t* counts,
+                           float* scores_out, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  return sa_select_blocks_gqa(L, Q, K, B, H, H, d, density, head_mask, min_active, idx, counts, scores_out, ws,
+                              ws_bytes, stream);
+}
+
+sa_status sa_select_blocks_noalloc_gqa(const sa_layout* L, const void* Q, const void* K, int B, int H, int H_kv,
+                                       int d, float density, const uint8_t* head_mask, int min_active, int32_t* idx,
+                                       int32_t* counts, float* scores_out, sa_stream_t stream) {
   if (!L || !Q || !K || !idx || !counts) return SA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K)) return SA_ERR_INVALID_ARG;
-  if (B <= 0 || (d != 64 && d != 128)) return SA_ERR_SHAPE;
+  if (B <= 0 || (d != 64 && d != 128) || !kv_heads_ok(H, H_kv)) return SA_ERR_SHAPE;
   if (static_cast<long long>(B) * H * L->N >= (1ll << 31)) return SA_ERR_SHAPE;
   if (!density_ok(density)) return SA_ERR_INVALID_ARG;
   uint64_t bits = 0;
@@ -302,8 +312,15 @@ sa_status sa_select_blocks_noalloc(const sa_layout* L, const void* Q, const void
   if ((st = check_device(&di)) != SA_OK) return st;
   if (di.id != L->device) return SA_ERR_INVALID_ARG;
   const int k = sa_budget(density, L->n_cand);
-  return from_cuda(launch_select_noalloc(L, Q, K, B, H, d, k, bits, idx, counts, scores_out,
+  return from_cuda(launch_select_noalloc(L, Q, K, B, H, H_kv, d, k, bits, idx, counts, scores_out,
                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_select_blocks_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int d,
+                                   float density, const uint8_t* head_mask, int min_active, int32_t* idx,
+                                   int32_t* counts, float* scores_out, sa_stream_t stream) {
+  return sa_select_blocks_noalloc_gqa(L, Q, K, B, H, H, d, density, head_mask, min_active, idx, counts, scores_out,
+                                      stream);
 }
 
 sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H, float density,
@@ -327,11 +344,11 @@ sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H,
                                   reinterpret_cast<cudaStream_t>(stream)));
 }
 
-static sa_status attention_args_ok(const void* Q, const void* K, const void* V, const void* O, int B, int H, int N,
-                                   int d, float* scale) {
+static sa_status attention_args_ok(const void* Q, const void* K, const void* V, const void* O, int B, int H,
+                                   int H_kv, int N, int d, float* scale) {
   if (!Q || !K || !V || !O) return SA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SA_ERR_INVALID_ARG;
-  if (B <= 0 || H <= 0 || H > kMaxHeads || (d != 64 && d != 128)) return SA_ERR_SHAPE;
+  if (B <= 0 || H <= 0 || H > kMaxHeads || (d != 64 && d != 128) || !kv_heads_ok(H, H_kv)) return SA_ERR_SHAPE;
   if (N <= 0 || N % kBlock || N / kBlock > kMaxBlocks) return SA_ERR_SHAPE;
   if (static_cast<long long>(B) * H * N >= (1ll << 31)) return SA_ERR_SHAPE;
   if (!std::isfinite(*scale) || *scale < 0.f) return SA_ERR_INVALID_ARG;
@@ -356,40 +373,60 @@ sa_status sa_attention_plan(const int32_t* idx, const int32_t* counts, int B, in
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
-sa_status sa_attention_run(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
-                           const uint8_t* head_mask, int min_active, float softmax_scale, void* O, void* ws,
-                           size_t ws_bytes, sa_stream_t stream) {
-  sa_status st = attention_args_ok(Q, K, V, O, B, H, N, d, &softmax_scale);
+sa_status sa_attention_run_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N, int d,
+                               const uint8_t* head_mask, int min_active, float softmax_scale, void* O, void* ws,
+                               size_t ws_bytes, sa_stream_t stream) {
+  sa_status st = attention_args_ok(Q, K, V, O, B, H, H_kv, N, d, &softmax_scale);
   if (st != SA_OK) return st;
   uint64_t bits = 0;
   if ((st = head_bits_of(head_mask, H, min_active, &bits)) != SA_OK) return st;
   if ((st = ws_ok(ws, ws_bytes, B, H, N, d)) != SA_OK) return st;
   DeviceInfo di;
   if ((st = check_device(&di)) != SA_OK) return st;
-  return from_cuda(launch_attention_run(Q, K, V, B, H, N, d, bits, softmax_scale, O, ws,
+  return from_cuda(launch_attention_run(Q, K, V, B, H, H_kv, N, d, bits, softmax_scale, O, ws,
                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_attention_run(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                           const uint8_t* head_mask, int min_active, float softmax_scale, void* O, void* ws,
+                           size_t ws_bytes, sa_stream_t stream) {
+  return sa_attention_run_gqa(Q, K, V, B, H, H, N, d, head_mask, min_active, softmax_scale, O, ws, ws_bytes, stream);
+}
+
+sa_status sa_block_sparse_attention_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N,
+                                        int d, const int32_t* idx, const int32_t* counts, int cap,
+                                        const uint8_t* head_mask, int min_active, float softmax_scale, void* O,
+                                        void* ws, size_t ws_bytes, sa_stream_t stream) {
+  sa_status st = attention_args_ok(Q, K, V, O, B, H, H_kv, N, d, &softmax_scale);
+  if (st != SA_OK) return st;
+  if ((st = sa_attention_plan(idx, counts, B, H, N, d, cap, head_mask, min_active, ws, ws_bytes, stream)) != SA_OK)
+    return st;
+  return sa_attention_run_gqa(Q, K, V, B, H, H_kv, N, d, head_mask, min_active, softmax_scale, O, ws, ws_bytes,
+                              stream);
 }
 
 sa_status sa_block_sparse_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
                                     const int32_t* idx, const int32_t* counts, int cap, const uint8_t* head_mask,
                                     int min_active, float softmax_scale, void* O, void* ws, size_t ws_bytes,
                                     sa_stream_t stream) {
-  sa_status st = attention_args_ok(Q, K, V, O, B, H, N, d, &softmax_scale);
-  if (st != SA_OK) return st;
-  if ((st = sa_attention_plan(idx, counts, B, H, N, d, cap, head_mask, min_active, ws, ws_bytes, stream)) != SA_OK)
-    return st;
-  return sa_attention_run(Q, K, V, B, H, N, d, head_mask, min_active, softmax_scale, O, ws, ws_bytes, stream);
+  return sa_block_sparse_attention_gqa(Q, K, V, B, H, H, N, d, idx, counts, cap, head_mask, min_active,
+                                       softmax_scale, O, ws, ws_bytes, stream);
 }
 
-sa_status sa_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
-                             float softmax_scale, void* O, void* ws, size_t ws_bytes, sa_stream_t stream) {
-  sa_status st = attention_args_ok(Q, K, V, O, B, H, N, d, &softmax_scale);
+sa_status sa_dense_attention_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N, int d,
+                                 float softmax_scale, void* O, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  sa_status st = attention_args_ok(Q, K, V, O, B, H, H_kv, N, d, &softmax_scale);
   if (st != SA_OK) return st;
   if (!ws || !aligned16(ws) || ws_bytes < sizeof(WsHeader)) return SA_ERR_WORKSPACE;
   DeviceInfo di;
   if ((st = check_device(&di)) != SA_OK) return st;
-  return from_cuda(launch_dense_attention(Q, K, V, B, H, N, d, softmax_scale, O, ws,
+  return from_cuda(launch_dense_attention(Q, K, V, B, H, H_kv, N, d, softmax_scale, O, ws,
                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+                             float softmax_scale, void* O, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  return sa_dense_attention_gqa(Q, K, V, B, H, H, N, d, softmax_scale, O, ws, ws_bytes, stream);
 }
 
 sa_status sa_density(const int32_t* counts, int B, int H, int nB, const uint8_t* head_mask, double* over_active,

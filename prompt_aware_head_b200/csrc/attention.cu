@@ -48,6 +48,7 @@ struct AttnArgs {
   int n_items_host;        // dense mode: item count
   int dense;               // 1: implicit full lists, pairs (2m, 2m+1)
   int N, nB, npairs_dense;
+  int H, g;                // query heads; query heads per key/value head (K and V hold B H / g heads)
   __nv_bfloat16* O;
   float scale_log2;
   int* err;
@@ -393,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qb = t % QB;
         const uint32_t uq = t / QB;
         if (uq >= 1 && !mbar_wait(&q_empty[qb], (uq - 1) & 1, abort_flag, a.err, kBackoffNs)) { ok = false; break; }
-        const int row0 = it.bh * a.N;
+        const int row0 = it.bh * a.N, krow0 = kv_head(it.bh, a.H, a.g) * a.N;
         uint8_t* qdst = sm + S::kQ + qb * S::kTile;
         mbar_expect_tx(&q_full[qb], (it.i1 != kNoBlock ? 2u : 1u) * kTxBlock);
 #pragma unroll
@@ -419,8 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(&k_full[kst], nblk * kTxBlock);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_2d(kdst + c * S::kChunk, &tmK, 64 * c, row0 + 64 * j0, &k_full[kst]);
-            if (nblk == 2) tma_load_2d(kdst + c * S::kChunk + 8192, &tmK, 64 * c, row0 + 64 * j1, &k_full[kst]);
+            tma_load_2d(kdst + c * S::kChunk, &tmK, 64 * c, krow0 + 64 * j0, &k_full[kst]);
+            if (nblk == 2) tma_load_2d(kdst + c * S::kChunk + 8192, &tmK, 64 * c, krow0 + 64 * j1, &k_full[kst]);
           }
           k_phase[kst] = uk & 1;
         }
@@ -450,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = load_item(a, k);
         const int nsteps = (it.len + 1) >> 1;
         if (nsteps == 0) continue;
-        const int row0 = it.bh * a.N;
+        const int row0 = kv_head(it.bh, a.H, a.g) * a.N;  // of V
         uint32_t e0n = load_entry(a, it, 0);
         uint32_t e1n = it.len > 1 ? load_entry(a, it, 1) : 0u;
         for (int s = 0; s < nsteps; ++s, ++g) {
@@ -792,12 +793,12 @@ static bool make_map(CUtensorMap* map, const void* base, size_t rows, int d) {
 }
 
 template <int D>
-static cudaError_t launch_attn_kernel(const void* Q, const void* K, const void* V, int BH, int N,
+static cudaError_t launch_attn_kernel(const void* Q, const void* K, const void* V, int BH, int BHkv, int N,
                                       const AttnArgs& args, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
-  const size_t rows = static_cast<size_t>(BH) * N;
-  const bool v_ok = (D == 128) ? make_map_v3(&mv, V, rows, D) : make_map(&mv, V, rows, D);
-  if (!make_map(&mq, Q, rows, D) || !make_map(&mk, K, rows, D) || !v_ok) return cudaErrorInvalidValue;
+  const size_t rows = static_cast<size_t>(BH) * N, kv_rows = static_cast<size_t>(BHkv) * N;
+  const bool v_ok = (D == 128) ? make_map_v3(&mv, V, kv_rows, D) : make_map(&mv, V, kv_rows, D);
+  if (!make_map(&mq, Q, rows, D) || !make_map(&mk, K, kv_rows, D) || !v_ok) return cudaErrorInvalidValue;
   DeviceInfo di;
   cudaError_t e = device_info(&di);
   if (e != cudaSuccess) return e;
@@ -810,13 +811,13 @@ static cudaError_t launch_attn_kernel(const void* Q, const void* K, const void* 
   return launch_pdl(sparse_attn_kernel<D>, dim3(di.sm_count), dim3(kThreads), AttnSmem<D>::kAlloc, s, mq, mk, mv, args);
 }
 
-static cudaError_t launch_attn(const void* Q, const void* K, const void* V, int BH, int N, int d,
+static cudaError_t launch_attn(const void* Q, const void* K, const void* V, int BH, int BHkv, int N, int d,
                                const AttnArgs& args, cudaStream_t s) {
-  if (d == 128) return launch_attn_kernel<128>(Q, K, V, BH, N, args, s);
-  return launch_attn_kernel<64>(Q, K, V, BH, N, args, s);
+  if (d == 128) return launch_attn_kernel<128>(Q, K, V, BH, BHkv, N, args, s);
+  return launch_attn_kernel<64>(Q, K, V, BH, BHkv, N, args, s);
 }
 
-cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int Hkv, int N, int d,
                                  uint64_t head_bits, float scale, void* O, void* ws, cudaStream_t s) {
   const int BH = B * H, nB = N / kBlock;
   const WsLayout wl = ws_layout(B, H, N, d);
@@ -838,14 +839,16 @@ cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, in
   args.N = N;
   args.nB = nB;
   args.npairs_dense = (nB + 1) / 2;
+  args.H = H;
+  args.g = H / Hkv;
   args.O = static_cast<__nv_bfloat16*>(O);
   args.scale_log2 = scale * 1.4426950408889634f;
   args.err = &hdr->err;
-  return launch_attn(Q, K, V, BH, N, d, args, s);
+  return launch_attn(Q, K, V, BH, B * Hkv, N, d, args, s);
 }
 
-cudaError_t launch_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
-                                   float scale, void* O, void* ws, cudaStream_t s) {
+cudaError_t launch_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int Hkv, int N,
+                                   int d, float scale, void* O, void* ws, cudaStream_t s) {
   const int BH = B * H, nB = N / kBlock;
   WsHeader* hdr = static_cast<WsHeader*>(ws);
   AttnArgs args{};
@@ -857,10 +860,12 @@ cudaError_t launch_dense_attention(const void* Q, const void* K, const void* V, 
   args.dense = 1;
   args.N = N;
   args.nB = nB;
+  args.H = H;
+  args.g = H / Hkv;
   args.O = static_cast<__nv_bfloat16*>(O);
   args.scale_log2 = scale * 1.4426950408889634f;
   args.err = &hdr->err;
-  return launch_attn(Q, K, V, BH, N, d, args, s);
+  return launch_attn(Q, K, V, BH, B * Hkv, N, d, args, s);
 }
 
 }  // namespace sa

@@ -19,6 +19,11 @@ enum BlockClass : uint8_t { kPin = 0, kSparse = 1, kDrop = 2 };
 // Attention work items and union lists mark "no second query block" with this.
 constexpr int kNoBlock = 0xFFFF;
 
+// Key/value head of query head bh = b H + h when groups of g consecutive
+// query heads share one (grouped-query attention): b (H / g) + h / g; g = 1
+// gives bh itself.
+__device__ __forceinline__ int kv_head(int bh, int H, int g) { return (bh / H) * (H / g) + (bh % H) / g; }
+
 // Error bits in the workspace header (mapped to sa_status by the host).
 enum ErrBits : int { kErrBadIndex = 1, kErrTimeout = 2, kErrSmemAlign = 4 };
 

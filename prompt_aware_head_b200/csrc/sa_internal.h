@@ -58,14 +58,15 @@ struct DeviceInfo {
 };
 cudaError_t device_info(DeviceInfo* out);
 
-// Selection / pattern / density launchers (select.cu).
-cudaError_t launch_select(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, int k,
+// Selection / pattern / density launchers (select.cu).  Hkv: key heads (H a
+// multiple of Hkv; query head b H + h scores against key head b Hkv + h / (H / Hkv)).
+cudaError_t launch_select(const sa_layout* L, const void* Q, const void* K, int B, int H, int Hkv, int d, int k,
                           uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out, void* ws,
                           cudaStream_t s);
 // Selection with its scratch in a fixed device array (no workspace).
 size_t select_noalloc_limit();
-cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, int k,
-                                  uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out,
+cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int Hkv, int d,
+                                  int k, uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out,
                                   cudaStream_t s);
 // kind: 0 radial, 1 window+global, 2 dilated, 3 dense (every non-drop block).
 cudaError_t launch_pattern(const sa_layout* L, int kind, int W, int G, int r, int k, int B, int H,
@@ -76,10 +77,10 @@ cudaError_t launch_density(const int32_t* counts, int B, int H, int nB, uint64_t
 // Work plan (plan.cu) and attention launchers (attention.cu).
 cudaError_t launch_attention_plan(const int32_t* idx, const int32_t* counts, int B, int H, int N, int d, int cap,
                                   uint64_t head_bits, void* ws, cudaStream_t s);
-cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
+cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int Hkv, int N, int d,
                                  uint64_t head_bits, float scale, void* O, void* ws, cudaStream_t s);
-cudaError_t launch_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
-                                   float scale, void* O, void* ws, cudaStream_t s);
+cudaError_t launch_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int Hkv, int N,
+                                   int d, float scale, void* O, void* ws, cudaStream_t s);
 
 cudaError_t launch_exp2_poly(const float* y, float* out, int n, cudaStream_t s);
 

@@ -329,12 +329,14 @@ __device__ __forceinline__ size_t img_offset(int i, int col) {
 // of Q and K.  16-byte vector loads, fp32 sums in a fixed order (per-thread
 // rows, then row groups in order), scaled by 1/64 (exact), then split into
 // hi / lo and written to the images of slot (RT row tiles per head).
-// HBM-bound.
-template <int D>
+// HBM-bound.  GQA (g query heads per key head): the key images are indexed
+// by key head, kv_head(bh) - kv0, and only the first active query head of a
+// group among this launch's heads pools the shared key head.
+template <int D, bool GQA>
 __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restrict__ Q,
                                                    const __nv_bfloat16* __restrict__ K, float* __restrict__ qimg,
                                                    float* __restrict__ kimg, int N, int nB, int RT, int H,
-                                                   uint64_t head_bits, int bh0, size_t lo_offset) {
+                                                   uint64_t head_bits, int bh0, size_t lo_offset, int g, int kv0) {
   grid_dep_wait();
   const int i = blockIdx.x, slot = blockIdx.y, bh = bh0 + slot;
   if (!((head_bits >> (bh % H)) & 1ull)) return;
@@ -342,15 +344,23 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
   constexpr int RG = 128 / TPR;  // row groups
   constexpr int RPT = 64 / RG;   // rows per thread
   const int t = threadIdx.x, cg = t % TPR, rg = t / TPR;
+  int kvh = bh;
+  bool pool_k = true;
+  if (GQA) {
+    kvh = kv_head(bh, H, g);
+    for (int h2 = max(bh - (bh % H) % g, bh0); h2 < bh; ++h2)
+      if ((head_bits >> (h2 % H)) & 1ull) pool_k = false;
+  }
   const size_t base = (static_cast<size_t>(bh) * N + static_cast<size_t>(i) * kBlock) * D;
+  const size_t kbase = (static_cast<size_t>(kvh) * N + static_cast<size_t>(i) * kBlock) * D;
   const uint4* q4 = reinterpret_cast<const uint4*>(Q + base);
-  const uint4* k4 = reinterpret_cast<const uint4*>(K + base);
+  const uint4* k4 = reinterpret_cast<const uint4*>(K + kbase);
   uint4 qv[RPT], kv[RPT];
 #pragma unroll
   for (int r = 0; r < RPT; ++r) {
     const int row = rg + r * RG;
     qv[r] = __ldg(q4 + row * TPR + cg);
-    kv[r] = __ldg(k4 + row * TPR + cg);
+    kv[r] = pool_k ? __ldg(k4 + row * TPR + cg) : make_uint4(0, 0, 0, 0);
   }
   float aq[8], ak[8];
 #pragma unroll
@@ -375,14 +385,15 @@ __global__ void __launch_bounds__(128) pool_kernel(const __nv_bfloat16* __restri
   }
   __syncthreads();
   const size_t head = static_cast<size_t>(slot) * RT * (D / 32) * kImgFloats;
-  for (int c = t; c < 2 * D; c += 128) {
+  const size_t khead = GQA ? static_cast<size_t>(kvh - kv0) * RT * (D / 32) * kImgFloats : head;
+  for (int c = t; c < (pool_k ? 2 : 1) * D; c += 128) {
     const int which = c / D, col = c % D;
     float s = 0.f;
 #pragma unroll
-    for (int g = 0; g < RG; ++g) s += red[which][g][col];
+    for (int rgi = 0; rgi < RG; ++rgi) s += red[which][rgi][col];
     s *= (1.0f / 64.0f);
     const float hi = tf32_rn(s);
-    float* img = (which ? kimg : qimg) + head + img_offset<D>(i, col);
+    float* img = (which ? kimg + khead : qimg + head) + img_offset<D>(i, col);
     img[0] = hi;
     img[lo_offset] = s - hi;
   }
@@ -411,6 +422,7 @@ struct TcArgs {
   int* err;
   size_t lo_offset;
   int nB, RT, H, bh0;
+  int g, kv0;     // query heads per key head; key head of bh0 (key images are indexed from it)
   int tma_store;  // 1: scores leave through the tensor map (3D [slot][nB][nB] fp32, 128-byte swizzle)
   uint64_t head_bits;
 };
@@ -485,7 +497,7 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(const __grid_constant_
   if (t == 0) {
     const size_t head = static_cast<size_t>(slot) * RT * NKC * kImgFloats;
     const float* qh = a.qimg + head;
-    const float* kh = a.kimg + head;
+    const float* kh = a.kimg + static_cast<size_t>(kv_head(bh, a.H, a.g) - a.kv0) * RT * NKC * kImgFloats;
     const uint32_t bytes = static_cast<uint32_t>((2 + 2 * nbt) * kImgBytes);
     auto load = [&](int kc, int s) {
       unsigned char* st = sm + s * kTcStage;
@@ -840,7 +852,7 @@ static size_t img_floats(int nB, int d) { return static_cast<size_t>((nB + kTcM 
 // The three kernels over heads bh0 .. bh0 + nbh - 1: the images (q, k: hi
 // then lo, nbh heads each) and scores are slot-indexed ([bh - bh0] ...),
 // idx / counts indexed by bh.
-static cudaError_t select_heads(const sa_layout* L, const void* Q, const void* K, int H, int d, int k,
+static cudaError_t select_heads(const sa_layout* L, const void* Q, const void* K, int H, int Hkv, int d, int k,
                                 uint64_t head_bits, int bh0, int nbh, float* qimg, float* kimg, float* scores, int* err,
                                 int32_t* idx, int32_t* counts, cudaStream_t s) {
   static bool configured[2][64];  // per head size, per device
@@ -856,15 +868,25 @@ static cudaError_t select_heads(const sa_layout* L, const void* Q, const void* K
   const size_t lo = static_cast<size_t>(nbh) * img_floats(nB, d);
   const auto* q = static_cast<const __nv_bfloat16*>(Q);
   const auto* kk = static_cast<const __nv_bfloat16*>(K);
-  e = d == 128 ? launch_pdl(pool_kernel<128>, dim3(nB, nbh), dim3(128), 0, s, q, kk, qimg, kimg, L->N, nB, RT, H,
-                            head_bits, bh0, lo)
-               : launch_pdl(pool_kernel<64>, dim3(nB, nbh), dim3(128), 0, s, q, kk, qimg, kimg, L->N, nB, RT, H,
-                            head_bits, bh0, lo);
+  // Key images are indexed by key head from kv0, the key head of bh0; the
+  // key heads of bh0 .. bh0 + nbh - 1 are consecutive, at most nbh of them.
+  const int g = H / Hkv, kv0 = (bh0 / H) * Hkv + (bh0 % H) / g;
+  const dim3 pg(nB, nbh);
+  if (g == 1)
+    e = d == 128 ? launch_pdl(pool_kernel<128, false>, pg, dim3(128), 0, s, q, kk, qimg, kimg, L->N, nB, RT, H,
+                              head_bits, bh0, lo, g, kv0)
+                 : launch_pdl(pool_kernel<64, false>, pg, dim3(128), 0, s, q, kk, qimg, kimg, L->N, nB, RT, H,
+                              head_bits, bh0, lo, g, kv0);
+  else
+    e = d == 128 ? launch_pdl(pool_kernel<128, true>, pg, dim3(128), 0, s, q, kk, qimg, kimg, L->N, nB, RT, H,
+                              head_bits, bh0, lo, g, kv0)
+                 : launch_pdl(pool_kernel<64, true>, pg, dim3(128), 0, s, q, kk, qimg, kimg, L->N, nB, RT, H,
+                              head_bits, bh0, lo, g, kv0);
   if (e != cudaSuccess) return e;
   CUtensorMap ms;
   std::memset(&ms, 0, sizeof ms);
   const int tma_store = make_score_map(&ms, scores, nB, nbh) ? 1 : 0;  // else plain row stores
-  TcArgs ta{qimg, kimg, scores, err, lo, nB, RT, H, bh0, tma_store, head_bits};
+  TcArgs ta{qimg, kimg, scores, err, lo, nB, RT, H, bh0, g, kv0, tma_store, head_bits};
   const dim3 grid((nB + kTcN - 1) / kTcN, RT, nbh);
   e = d == 128 ? launch_pdl(score_tc_kernel<128>, grid, dim3(128), kTcSmem, s, ta, ms)
                : launch_pdl(score_tc_kernel<64>, grid, dim3(128), kTcSmem, s, ta, ms);
@@ -872,7 +894,7 @@ static cudaError_t select_heads(const sa_layout* L, const void* Q, const void* K
   return launch_rank(nc, scores, L, bh0, nbh, H, head_bits, k, idx, counts, s);
 }
 
-cudaError_t launch_select(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, int k,
+cudaError_t launch_select(const sa_layout* L, const void* Q, const void* K, int B, int H, int Hkv, int d, int k,
                           uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out, void* ws,
                           cudaStream_t s) {
   if (k >= L->n_cand && scores_out == nullptr)  // the budget covers every candidate: dense lists, no scoring
@@ -880,7 +902,7 @@ cudaError_t launch_select(const sa_layout* L, const void* Q, const void* K, int 
   const WsLayout wl = ws_layout(B, H, L->N, d);
   char* base = static_cast<char*>(ws);
   float* scores = scores_out ? scores_out : reinterpret_cast<float*>(base + wl.scores);
-  return select_heads(L, Q, K, H, d, k, head_bits, 0, B * H, reinterpret_cast<float*>(base + wl.qbar),
+  return select_heads(L, Q, K, H, Hkv, d, k, head_bits, 0, B * H, reinterpret_cast<float*>(base + wl.qbar),
                       reinterpret_cast<float*>(base + wl.kbar), scores,
                       &reinterpret_cast<WsHeader*>(base + wl.header)->err, idx, counts, s);
 }
@@ -917,8 +939,8 @@ static cudaError_t noalloc_scratch(void** out) {
   return cudaSuccess;
 }
 
-cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int d, int k,
-                                  uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out,
+cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int Hkv, int d,
+                                  int k, uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out,
                                   cudaStream_t s) {
   const int BH = B * H, nB = L->nB;
   if (k >= L->n_cand && scores_out == nullptr)  // dense lists: no scratch used
@@ -942,7 +964,7 @@ cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void*
   for (int bh0 = 0; bh0 < BH; bh0 += G) {
     const int nbh = std::min(G, BH - bh0);
     float* sc = scores_out ? scores_out + static_cast<size_t>(bh0) * nB * nB : sc_scratch;
-    e = select_heads(L, Q, K, H, d, k, head_bits, bh0, nbh, qimg, kimg, sc, err, idx, counts, s);
+    e = select_heads(L, Q, K, H, Hkv, d, k, head_bits, bh0, nbh, qimg, kimg, sc, err, idx, counts, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -85,3 +85,15 @@ def test_argument_checks_before_any_launch(lib):
         lib.sa_block_sparse_attention(fake, fake, fake, 1, 4, 512, 64, fake, fake, 8, None, 0, -1.0, fake,
                                       fake, 1 << 30, stream=0)
     assert e.value.status == lib.SA_ERR_INVALID_ARG     # negative softmax scale
+
+
+def test_grouped_head_counts_checked_before_any_launch(lib):
+    fake = 1 << 20
+    for H_kv in (0, 4, 12):  # 6 query heads: no key heads, a partial group, more key than query heads
+        with pytest.raises(lib.SAError) as e:
+            lib.sa_dense_attention_gqa(fake, fake, fake, 1, 6, H_kv, 512, 64, 0.0, fake, fake, 1 << 20, stream=0)
+        assert e.value.status == lib.SA_ERR_SHAPE
+        with pytest.raises(lib.SAError) as e:
+            lib.sa_block_sparse_attention_gqa(fake, fake, fake, 1, 6, H_kv, 512, 64, fake, fake, 8, None, 0, 0.0,
+                                              fake, fake, 1 << 30, stream=0)
+        assert e.value.status == lib.SA_ERR_SHAPE
