@@ -26,7 +26,7 @@
  *          (attend to all, attended by all), block-sparse (only connected
  *          block pairs computed).
  *
- * Readings where the pages are silent (each listed in the design doc):
+ * Readings where the pages are silent (the CUDA library takes the same ones):
  *   budget k = clamp(floor(rho*C + 1e-4), 1, C) with C the sparsifiable
  *   candidates; the diagonal is forced and counts in k; ties break to the
  *   lower block index; -0 ranks as +0; lists are emitted in ascending block

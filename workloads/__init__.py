@@ -5,7 +5,7 @@ tests.  It holds none of the method's arithmetic: it only draws random
 numbers, rounds them to bf16, and describes the workloads (shapes, token
 segments, head masks, density budgets).
 
-Recipe (also stated in the design doc):
+Recipe:
   rng = numpy.random.default_rng([seed, layer, tensor_id]) with tensor_id
   Q=0, K=1, V=2, P=3, head-mask=4.
   V ~ N(0, 1).
