@@ -1,0 +1,80 @@
+"""bench.py on the CPU: the reference arm's JSON line and the host helpers.
+
+The reference arm times the fp64 oracle on the host cores; on the tiny
+workload it finishes in seconds.  Nothing here touches a GPU.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from workloads import WORKLOADS, make_qkv  # noqa: E402
+
+
+def _reference_line(*extra):
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                          "--steps", "1", "--warmup", "3", *extra], capture_output=True, text=True, env=env,
+                         timeout=600, check=True)
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1, out.stdout
+    return json.loads(lines[0])
+
+
+@pytest.mark.parametrize("extra", [(), ("--kv-heads", "2")])
+def test_reference_arm_line(extra):
+    d = _reference_line(*extra)
+    assert d["impl"] == "reference"
+    assert d["metric"] == bench.METRIC and d["unit"] == bench.UNIT and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 3
+    assert d["dtype"] == "f64"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["H_kv"] == (2 if extra else 4)
+    assert d["config"]["workload"].startswith("tiny: B1 H4")
+
+
+def test_reference_arm_other_ranks_print_nothing():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                          "--steps", "1", "--warmup", "3"], capture_output=True, text=True, env=env, timeout=600,
+                         check=True)
+    assert out.stdout.strip() == ""
+
+
+def test_bad_kv_heads_rejected():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                          "--steps", "1", "--warmup", "3", "--kv-heads", "3"], capture_output=True, text=True, env=env,
+                         timeout=600)
+    assert out.returncode != 0 and "kv-heads" in out.stderr
+
+
+def test_grouped_kv_takes_each_groups_first_head():
+    w = WORKLOADS["tiny"]
+    _, K, V = make_qkv(w)
+    Kg, Vg = bench.grouped_kv(K, V, 2)
+    assert Kg.shape == (1, 2, w.N, w.d) and Kg.flags.c_contiguous
+    np.testing.assert_array_equal(Kg[:, 1], K[:, 2])
+    np.testing.assert_array_equal(Vg[:, 0], V[:, 0])
+
+
+def test_describe_names_grouped_heads():
+    w = WORKLOADS["joint"]
+    assert "(K/V heads 6)" in bench.describe(w, 0.3, 6)
+    assert "K/V heads" not in bench.describe(w, 0.3, 24)
+    assert "K/V heads" not in bench.describe(w, 0.3)
+
+
+def test_traffic_is_null_when_the_kernel_source_differs(tmp_path):
+    src = tmp_path / "attention.cu"
+    src.write_text("// not the profiled kernel\n")
+    assert bench.traffic_from_profile(str(src)) is None
