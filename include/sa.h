@@ -137,6 +137,33 @@ SA_API sa_status sa_layout_release(sa_layout* L);
 SA_API int sa_budget(float density, int n_cand);
 
 /*
+ * Per-step budgets [SDN stage paragraph: budgets follow a precomputed
+ * per-step schedule with at most two distinct values].  Checks a schedule
+ * of n_steps densities, each finite and in (0, 1], with at most two distinct
+ * values, and writes for step t:
+ *   k_out[t]     = sa_budget(densities[t], n_cand);
+ *   dense_out[t] = 1 when k_out[t] == n_cand (the selection then writes
+ *                  dense lists without pooling or scoring), else 0.
+ * Either output may be NULL.  Host memory only; no device is touched.
+ * SA_ERR_INVALID_ARG for NULL densities, n_steps < 1, n_cand < 1, a density
+ * outside (0, 1], or a third distinct value (nothing is written then).
+ */
+SA_API sa_status sa_budget_schedule(const float* densities, int n_steps, int n_cand, int32_t* k_out,
+                                    uint8_t* dense_out);
+
+/*
+ * Whether a call takes the block-sparse path [SDN stage paragraph: the
+ * stage gates on self attention, a minimum sequence length (8192 tokens by
+ * default, the sparse/dense crossover measured there), and the absence of a
+ * token mask or causal flag, which a block-only mask cannot combine with].
+ * Returns 1 when is_self_attention != 0, has_token_mask == 0, is_causal == 0
+ * and N >= min_seq_len (min_seq_len <= 0 means SA_DEFAULT_MIN_SEQ_LEN),
+ * else 0 (stay dense).  Host only.
+ */
+#define SA_DEFAULT_MIN_SEQ_LEN 8192
+SA_API int sa_sparse_stage_gate(int N, int min_seq_len, int is_self_attention, int has_token_mask, int is_causal);
+
+/*
  * sa_select_blocks [SDN "selector" + "host sync" paragraphs].
  * Per (batch, active head, 64-row query block i):
  *   qbar_i = mean of the 64 Q rows, kbar_j likewise (fp32 accumulation);

@@ -7,7 +7,7 @@ sa_pattern_mask, sa_block_sparse_attention, sa_dense_attention, sa_density,
 (int); PyTorch is used only to hold device memory and streams.
 
 Importing this module raises if the compiled library is missing: there is no
-fallback path.  Build it with ``python -m prompt_aware_head_b200.build`` (or
+fallback path.  Build it with ``python prompt_aware_head_b200/build.py`` (or
 ``__graft_entry__.build()``).
 """
 from __future__ import annotations
@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libsa_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("libsa_b200.so not found at %s: build the CUDA library first "
-                      "(python -m prompt_aware_head_b200.build)" % LIB_PATH)
+                      "(python prompt_aware_head_b200/build.py)" % LIB_PATH)
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -38,6 +38,7 @@ SA_PAT_RADIAL, SA_PAT_WINDOW_GLOBAL, SA_PAT_DILATED = range(3)
 # per layer and the default fraction of heads to skip.
 MIN_ACTIVE_HEADS = 4
 DEFAULT_SPARSITY = 0.5
+DEFAULT_MIN_SEQ_LEN = 8192  # SA_DEFAULT_MIN_SEQ_LEN
 
 
 class sa_segment(ctypes.Structure):
@@ -61,6 +62,8 @@ _SIGS = {
     "sa_layout_classes": ([_P, _P, _I], _I),
     "sa_layout_release": ([_P], _I),
     "sa_budget": ([_F, _I], _I),
+    "sa_budget_schedule": ([_P, _I, _I, _P, _P], _I),
+    "sa_sparse_stage_gate": ([_I, _I, _I, _I, _I], _I),
     "sa_select_blocks": ([_P, _P, _P, _I, _I, _I, _F, _P, _I, _P, _P, _P, _P, _SZ, _P], _I),
     "sa_select_blocks_noalloc": ([_P, _P, _P, _I, _I, _I, _F, _P, _I, _P, _P, _P, _P], _I),
     "sa_pattern_mask": ([_P, ctypes.POINTER(sa_pattern), _I, _I, _F, _P, _I, _P, _P, _P], _I),
@@ -163,6 +166,25 @@ def sa_build_layout(segments, N: int, block: int = 64) -> Layout:
 
 def sa_budget(density: float, n_cand: int) -> int:
     return int(_lib.sa_budget(ctypes.c_float(density), int(n_cand)))
+
+
+def sa_budget_schedule(densities, n_cand: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-step budgets k and dense flags of a schedule with at most two
+    distinct densities (host only)."""
+    d = np.ascontiguousarray(densities, dtype=np.float32).reshape(-1)
+    k = np.zeros(d.size, dtype=np.int32)
+    dense = np.zeros(d.size, dtype=np.uint8)
+    _check(_lib.sa_budget_schedule(d.ctypes.data_as(ctypes.c_void_p), int(d.size), int(n_cand),
+                                   k.ctypes.data_as(ctypes.c_void_p), dense.ctypes.data_as(ctypes.c_void_p)),
+           "sa_budget_schedule")
+    return k, dense.astype(bool)
+
+
+def sa_sparse_stage_gate(N: int, min_seq_len: int = 0, self_attention: bool = True, token_mask: bool = False,
+                         causal: bool = False) -> bool:
+    """True when a call should take the block-sparse path (host only)."""
+    return bool(_lib.sa_sparse_stage_gate(int(N), int(min_seq_len), int(bool(self_attention)), int(bool(token_mask)),
+                                          int(bool(causal))))
 
 
 def sa_workspace_size(B: int, H: int, N: int, d: int) -> int:

@@ -134,6 +134,32 @@ int sa_budget(float density, int n_cand) {
   return static_cast<int>(k);
 }
 
+sa_status sa_budget_schedule(const float* densities, int n_steps, int n_cand, int32_t* k_out, uint8_t* dense_out) {
+  if (!densities || n_steps < 1 || n_cand < 1) return SA_ERR_INVALID_ARG;
+  float seen[2];
+  int n_seen = 0;
+  for (int t = 0; t < n_steps; ++t) {
+    const float r = densities[t];
+    if (!density_ok(r)) return SA_ERR_INVALID_ARG;
+    bool known = false;
+    for (int v = 0; v < n_seen; ++v) known = known || seen[v] == r;
+    if (known) continue;
+    if (n_seen == 2) return SA_ERR_INVALID_ARG;
+    seen[n_seen++] = r;
+  }
+  for (int t = 0; t < n_steps; ++t) {
+    const int k = sa_budget(densities[t], n_cand);
+    if (k_out) k_out[t] = k;
+    if (dense_out) dense_out[t] = k == n_cand ? 1 : 0;
+  }
+  return SA_OK;
+}
+
+int sa_sparse_stage_gate(int N, int min_seq_len, int is_self_attention, int has_token_mask, int is_causal) {
+  const int min_len = min_seq_len > 0 ? min_seq_len : SA_DEFAULT_MIN_SEQ_LEN;
+  return (is_self_attention && !has_token_mask && !is_causal && N >= min_len) ? 1 : 0;
+}
+
 sa_status sa_build_layout(const sa_segment* segs, int nseg, int N, int block, sa_layout** out) {
   if (!out || nseg < 0 || (nseg > 0 && !segs)) return SA_ERR_INVALID_ARG;
   if (block != kBlock || N <= 0 || N % block != 0 || N / block > kMaxBlocks) return SA_ERR_SHAPE;
