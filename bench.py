@@ -75,6 +75,15 @@ def max_over_ranks(x, device):
     return float(t.item())
 
 
+def time_stats(times_ms):
+    """Mean, median and 90th percentile (nearest rank) of per-step times, ms."""
+    xs = sorted(float(x) for x in times_ms)
+    if not xs:
+        raise ValueError("no times")
+    p90 = xs[max(0, -(-9 * len(xs) // 10) - 1)]
+    return {"mean": round(statistics.mean(xs), 5), "median": round(statistics.median(xs), 5), "p90": round(p90, 5)}
+
+
 def job_value(flops_per_rank, ms_max, world):
     """Whole-job effective TFLOP/s: every rank's flops over the slowest rank's
     time (each rank runs its own batch: weak scaling)."""
@@ -427,6 +436,8 @@ def run_ours(args):
         },
         "breakdown_ms": {"select": round(sel_ms, 5), "plan": round(statistics.mean(t_plan), 5),
                          "attention": round(att_ms, 5)},
+        "time_stats_ms": {"step": time_stats(t_step), "select": time_stats(t_sel), "plan": time_stats(t_plan),
+                          "attention": time_stats(t_att)},
         "speedup_vs_dense": round(dense_ms / ms_step, 3) if dense_ms else None,
         "attention_speedup_vs_dense": round(dense_ms / att_ms, 3) if dense_ms else None,
         "dense_ms": round(dense_ms, 5) if dense_ms else None,

@@ -78,3 +78,13 @@ def test_traffic_is_null_when_the_kernel_source_differs(tmp_path):
     src = tmp_path / "attention.cu"
     src.write_text("// not the profiled kernel\n")
     assert bench.traffic_from_profile(str(src)) is None
+
+
+def test_time_stats():
+    assert bench.time_stats([3.0]) == {"mean": 3.0, "median": 3.0, "p90": 3.0}
+    xs = [float(i) for i in range(1, 11)]             # 1 .. 10: nearest-rank p90 is the 9th value
+    assert bench.time_stats(xs[::-1]) == {"mean": 5.5, "median": 5.5, "p90": 9.0}
+    assert bench.time_stats(list(range(1, 21)))["p90"] == 18.0
+    assert bench.time_stats([1, 2, 3])["p90"] == 3.0
+    with pytest.raises(ValueError):
+        bench.time_stats([])
