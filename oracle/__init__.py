@@ -51,7 +51,7 @@ def _load():
         _lib.oracle_select.argtypes = [P, P, i, i, i, f, P, i, P, P]
         _lib.oracle_pattern.argtypes = [P, i, i, i, i, i, i, f, i, i, P, i, P, P]
         _lib.oracle_pattern.restype = i
-        _lib.oracle_attention.argtypes = [P, P, P, i, i, i, i, i, i, P, P, i, P, dbl, P, ctypes.c_int64, P]
+        _lib.oracle_attention.argtypes = [P, P, P, i, i, i, i, i, i, P, P, i, P, P, dbl, P, ctypes.c_int64, P]
         _lib.oracle_density.argtypes = [P, i, i, i, P, P, P]
     return _lib
 
@@ -155,13 +155,16 @@ def pattern(cls: np.ndarray, kind: int, BH: int, H: int, window: int = 0, n_glob
 
 def attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, H: int, idx: np.ndarray, counts: np.ndarray,
               head_mask: Optional[np.ndarray] = None, scale: Optional[float] = None,
-              rows: Optional[np.ndarray] = None, block: int = 64) -> np.ndarray:
+              rows: Optional[np.ndarray] = None, block: int = 64,
+              key_mask: Optional[np.ndarray] = None) -> np.ndarray:
     """fp64 attention over the kept tiles; Q uint16 bf16 bits [B, H, N, d],
     K and V [B, Hkv, N, d] with H a multiple of Hkv (query head h reads
     key/value head h // (H / Hkv)).
 
     rows: flat row ids (b*H + h)*N + n to compute (None = all); returns
-    [len(rows), d] (or [B, H, N, d] when rows is None)."""
+    [len(rows), d] (or [B, H, N, d] when rows is None).
+    key_mask: optional token-level mask over keys, [B, N] (nonzero = may be
+    attended), applied inside the kept tiles; a row left with no key gives 0."""
     lib = _load()
     Q = np.ascontiguousarray(Q, dtype=np.uint16)
     K = np.ascontiguousarray(K, dtype=np.uint16)
@@ -176,15 +179,20 @@ def attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, H: int, idx: np.ndarr
     cap = idx.shape[-1]
     hm = None if head_mask is None else np.ascontiguousarray(head_mask, dtype=np.uint8)
     sc = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    km = None
+    if key_mask is not None:
+        km = np.ascontiguousarray(np.asarray(key_mask) != 0, dtype=np.uint8)
+        if km.size != (BH // H) * N:
+            raise ValueError("key_mask must be [B, N]")
     if rows is None:
         out = np.zeros((BH * N, d), dtype=np.float64)
         lib.oracle_attention(_ptr(Q), _ptr(K), _ptr(V), BH, H, Hkv, N, d, block, _ptr(idx), _ptr(counts), cap,
-                             _ptr(hm), sc, None, BH * N, _ptr(out))
+                             _ptr(hm), _ptr(km), sc, None, BH * N, _ptr(out))
         return out.reshape(Q.shape)
     rows = np.ascontiguousarray(rows, dtype=np.int64)
     out = np.zeros((rows.shape[0], d), dtype=np.float64)
     lib.oracle_attention(_ptr(Q), _ptr(K), _ptr(V), BH, H, Hkv, N, d, block, _ptr(idx), _ptr(counts), cap,
-                         _ptr(hm), sc, _ptr(rows), rows.shape[0], _ptr(out))
+                         _ptr(hm), _ptr(km), sc, _ptr(rows), rows.shape[0], _ptr(out))
     return out
 
 

@@ -301,10 +301,14 @@ int oracle_pattern(const uint8_t* cls, int nB, int block, int kind, int W, int G
  * [BH][N][d]; K and V are [B*Hkv][N][d], query head bh reading key/value
  * head kv_head(bh); rows lists flat row ids bh*N + n (NULL = every row);
  * out is [nrows][d] fp64.
+ * key_mask (NULL = none) is a token-level mask over keys, [B][N] bytes, 1 =
+ * may be attended: a key inside a kept tile counts only where it is set
+ * [SDN "masked_block": a backend takes the attention mask and the block
+ * mask together].  A row none of whose kept keys is set gives O = 0.
  */
 void oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int BH, int H, int Hkv, int N, int d,
                       int block, const int32_t* idx, const int32_t* counts, int cap, const uint8_t* head_mask,
-                      double scale, const int64_t* rows, int64_t nrows, double* out) {
+                      const uint8_t* key_mask, double scale, const int64_t* rows, int64_t nrows, double* out) {
   int nB = N / block;
   if (!rows) nrows = (int64_t)BH * N;
 #pragma omp parallel
@@ -325,6 +329,15 @@ void oracle_attention(const uint16_t* Q, const uint16_t* K, const uint16_t* V, i
       const int32_t* li = idx + ((size_t)bh * nB + i) * cap;
       for (int e = 0; e < cnt; ++e)
         for (int r = 0; r < block; ++r) keep[(size_t)li[e] * block + r] = 1;
+      if (key_mask) {
+        const uint8_t* km = key_mask + (size_t)(bh / H) * N;
+        int any = 0;
+        for (int key = 0; key < N; ++key) {
+          keep[key] = keep[key] && km[key];
+          any |= keep[key];
+        }
+        if (!any) continue;
+      }
       for (int c = 0; c < d; ++c) q[c] = bf16_to_double(Q[((size_t)bh * N + n) * d + c]);
       double mx = -INFINITY;
       for (int key = 0; key < N; ++key) {

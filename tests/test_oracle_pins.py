@@ -396,3 +396,61 @@ def test_grouped_heads_reject_a_partial_group():
     q = np.zeros((1, 6, 2, 8))
     with pytest.raises(ValueError):
         oracle.scores(q, np.zeros((1, 4, 2, 8)))
+
+
+# ---------------------------------------------------------------- token-level key mask inside kept tiles
+
+def _key_mask_case(seed=12):
+    """Two batches of the tiny layout, each with its own live prompt length:
+    keys past the live text (inside the straddling pinned block) and the
+    padding are masked."""
+    w = WORKLOADS["tiny"]
+    rng = np.random.default_rng(seed)
+    B, H, N, d = 2, 2, w.N, w.d
+    Q, K, V = (_bits(rng.standard_normal((B, H, N, d))) for _ in range(3))
+    km = np.ones((B, N), np.uint8)
+    km[0, 25:128] = 0   # batch 0: 25 live text tokens
+    km[1, 40:128] = 0   # batch 1: 40
+    cls = oracle.layout(list(w.segments), N)
+    sc = oracle.scores(oracle.pool(Q), oracle.pool(K)).reshape(-1, w.nB, w.nB)
+    idx, counts = oracle.select(sc, cls, H, 0.5)
+    return w, Q, K, V, km, idx, counts
+
+
+def test_key_mask_equals_masked_sdpa():
+    w, Q, K, V, km, idx, counts = _key_mask_case()
+    B, H, N = Q.shape[0], Q.shape[1], w.N
+    got = oracle.attention(Q, K, V, H, idx, counts, key_mask=km)
+    tiles = _token_mask(idx.reshape(-1, w.nB, idx.shape[-1]), counts.reshape(-1, w.nB), N).reshape(B, H, N, N)
+    mask = tiles & (km[:, None, None, :] != 0)
+    live = mask.any(-1)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(_f64(x)) for x in (Q, K, V)), attn_mask=torch.from_numpy(mask)).numpy()
+    np.testing.assert_allclose(got[live], ref[live], rtol=1e-12, atol=1e-12)
+    assert np.all(got[~live] == 0)
+    # the two batches' masks differ: the result depends on each batch's own mask
+    swapped = oracle.attention(Q, K, V, H, idx, counts, key_mask=km[::-1].copy())
+    assert not np.allclose(swapped[0], got[0])
+
+
+def test_key_mask_of_ones_changes_nothing():
+    w, Q, K, V, _, idx, counts = _key_mask_case()
+    np.testing.assert_array_equal(oracle.attention(Q, K, V, 2, idx, counts, key_mask=np.ones((2, w.N), np.uint8)),
+                                  oracle.attention(Q, K, V, 2, idx, counts))
+
+
+def test_key_mask_closed_forms():
+    w, _, K, V, km, idx, counts = _key_mask_case()
+    B, H, N = K.shape[0], K.shape[1], w.N
+    out = oracle.attention(np.zeros_like(K), K, V, H, idx, counts, key_mask=km)
+    Vf = _f64(V)
+    for b, h, i in ((0, 0, 0), (1, 1, 0), (0, 1, 5), (1, 0, 7)):
+        keys = np.concatenate([np.arange(64 * j, 64 * j + 64) for j in idx[b * H + h, i, :counts[b * H + h, i]]])
+        keys = keys[km[b, keys] != 0]
+        np.testing.assert_allclose(out[b, h, 64 * i:64 * i + 64], np.broadcast_to(Vf[b, h, keys].mean(0), (64, w.d)),
+                                   rtol=1e-12, atol=1e-12)
+    # a row whose only kept tile is fully masked gives exact zeros
+    one_idx = np.full((B * H, w.nB, 1), 1, np.int32)
+    one_cnt = np.ones((B * H, w.nB), np.int32)
+    out = oracle.attention(_bits(np.ones((B, H, N, w.d))), K, V, H, one_idx, one_cnt, key_mask=km)
+    assert np.all(out == 0)
