@@ -102,6 +102,7 @@ def oracle_sample(w, rho, target_s=10.0, seed=0, g=1):
     cls = oracle.layout(list(w.segments), w.N)
     flops = 0.0
     t_total = 0.0
+    sel_s, att_s = 0.0, 0.0  # unscaled: every timed selection, every timed attention row
     done_heads, done_rows = 0, 0
     for h in heads:
         Q, K, V = make_qkv(w, seed=seed, heads=[h])
@@ -124,6 +125,8 @@ def oracle_sample(w, rho, target_s=10.0, seed=0, g=1):
         t = time.perf_counter()
         oracle.attention(Q, K, V, 1, idx, cnt, rows=rows)
         t_att = time.perf_counter() - t
+        sel_s += t_sel
+        att_s += t_att
         flops += float(np.sum(4.0 * w.d * 64 * cnt[0, rows // 64]))
         t_total += t_att + t_sel * len(rows) / w.N
         done_heads += 1
@@ -138,6 +141,8 @@ def oracle_sample(w, rho, target_s=10.0, seed=0, g=1):
         "kind": "oracle",
         "sample": "%d of %d heads of the workload: fp64 selection per head (charged pro rata to the rows run) + "
                   "fp64 attention for %d query rows in all (%.1f s)" % (done_heads, len(heads), done_rows, t_total),
+        "split": {"select_ms_per_head": round(1e3 * sel_s / max(done_heads, 1), 3),
+                  "attention_us_per_row": round(1e6 * att_s / max(done_rows, 1), 3)},
         "seconds": t_total,
     }
 
@@ -506,7 +511,7 @@ def run_reference(args):
         "config": {"workload": describe(w, rho, H_kv), "B": w.B, "H": w.H, "H_kv": H_kv, "N": w.N, "d": w.d,
                    "density_budget": rho},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last["cores"], "kind": "oracle",
-                         "sample": last["sample"]},
+                         "sample": last["sample"], "split": last["split"]},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
