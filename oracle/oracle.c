@@ -290,13 +290,13 @@ int oracle_pattern(const uint8_t* cls, int nB, int block, int kind, int W, int G
         } else if (kind == OR_PAT_RANDOM) {
           /* [GLO random: each query attends to a fixed set of keys sampled
            * uniformly at random]: the diagonal, then the k - 1 other sparse
-           * blocks ranked by the top 22 bits of output i*nB + j + 1, larger
+           * blocks ranked by the top 21 bits of output i*nB + j + 1, larger
            * first (ties: lower block), the same for every head */
           int nc = 0;
           for (int j = 0; j < nB; ++j) {
             if (cls[j] != OR_SPARSE) continue;
             cand[nc].key = (j == i) ? INFINITY
-                                    : (double)(splitmix64_nth(seed, (uint64_t)i * (uint64_t)nB + (uint64_t)j + 1) >> 42);
+                                    : (double)(splitmix64_nth(seed, (uint64_t)i * (uint64_t)nB + (uint64_t)j + 1) >> 43);
             cand[nc].j = j;
             ++nc;
           }
