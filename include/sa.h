@@ -329,6 +329,13 @@ SA_API const char* sa_status_string(sa_status s);
  * floats.  Not on the hot path; for tests. */
 SA_API sa_status sa_debug_exp2(const float* y, float* out, int n, sa_stream_t stream);
 
+/* Diagnostic: one kernel waits, through the same bounded-wait helper every
+ * kernel uses, on a barrier that nothing completes.  After the wait limit
+ * (2 s) it records SA_ERR_TIMEOUT in the workspace error word and returns,
+ * so the next sa_check reports SA_ERR_TIMEOUT and the device stays usable.
+ * Not on the hot path; for tests. */
+SA_API sa_status sa_debug_wait_timeout(void* ws, size_t ws_bytes, sa_stream_t stream);
+
 /* Library version string. */
 SA_API const char* sa_version(void);
 

@@ -82,6 +82,7 @@ _SIGS = {
     "sa_workspace_init": ([_P, _SZ, _P], _I),
     "sa_check": ([_P, _P], _I),
     "sa_debug_exp2": ([_P, _P, _I, _P], _I),
+    "sa_debug_wait_timeout": ([_P, _SZ, _P], _I),
     "sa_status_string": ([_I], ctypes.c_char_p),
     "sa_version": ([], ctypes.c_char_p),
 }
@@ -308,6 +309,12 @@ def sa_density(counts, B: int, H: int, nB: int, head_mask, ws, ws_bytes: int, st
     _check(_lib.sa_density(_addr(counts), B, H, nB, mptr, ctypes.byref(a), ctypes.byref(b), ctypes.byref(st),
                            _addr(ws), ws_bytes, _stream(stream)), "sa_density")
     return a.value, b.value, st
+
+
+def sa_debug_wait_timeout(ws, ws_bytes: int, stream=None) -> None:
+    """Runs one kernel whose bounded wait runs out (about 2 s); the next
+    sa_check reports SA_ERR_TIMEOUT."""
+    _check(_lib.sa_debug_wait_timeout(_addr(ws), ws_bytes, _stream(stream)), "sa_debug_wait_timeout")
 
 
 def sa_debug_exp2(y, out, n: int, stream=None) -> None:

@@ -39,6 +39,22 @@ WsLayout ws_layout(int B, int H, int N, int d) {
   return w;
 }
 
+// Diagnostic for the bounded waits: one thread waits, through the same
+// helper every kernel uses, on a shared-memory barrier that nothing arrives
+// at.  After the wait limit the helper records kErrTimeout in *err and the
+// kernel returns; nothing traps, and the context stays usable.
+__global__ void wait_timeout_kernel(int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, err);  // phase 0 never completes: runs out
+}
+
 cudaError_t device_info(DeviceInfo* out) {
   static DeviceInfo cache[64];
   static std::mutex mu;
@@ -481,6 +497,15 @@ sa_status sa_density(const int32_t* counts, int B, int H, int nB, const uint8_t*
     stats->heads_active = active;
   }
   return SA_OK;
+}
+
+sa_status sa_debug_wait_timeout(void* ws, size_t ws_bytes, sa_stream_t stream) {
+  if (!ws || !aligned16(ws) || ws_bytes < sizeof(WsHeader)) return SA_ERR_WORKSPACE;
+  DeviceInfo di;
+  sa_status st = check_device(&di);
+  if (st != SA_OK) return st;
+  wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(&static_cast<WsHeader*>(ws)->err);
+  return from_cuda(cudaGetLastError());
 }
 
 sa_status sa_debug_exp2(const float* y, float* out, int n, sa_stream_t stream) {
