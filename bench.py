@@ -274,7 +274,7 @@ def run_ours(args):
         raise SystemExit("--kv-heads must divide the workload's %d heads" % H)
     g = H // H_kv
     mask = head_mask_for_layer(w)
-    Qh, Kh, Vh = make_qkv(w, seed=rank)
+    Qh, Kh, Vh = make_qkv(w, seed=args.seed + rank)
     if g > 1:
         Kh, Vh = grouped_kv(Kh, Vh, g)
     pin = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (Qh, Kh, Vh)]
@@ -495,7 +495,7 @@ def run_ours(args):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = oracle_sample(w, rho, target_s=args.cpu_seconds, seed=rank, g=g)
+        cb = oracle_sample(w, rho, target_s=args.cpu_seconds, seed=args.seed + rank, g=g)
         cb.pop("seconds", None)
         out["cpu_baseline"] = cb
     if world > 1:
@@ -585,10 +585,10 @@ def run_reference(args):
     g = w.H // H_kv
     per_step = max(2.0, 120.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        oracle_sample(w, rho, target_s=min(per_step, 2.0), g=g)
+        oracle_sample(w, rho, target_s=min(per_step, 2.0), seed=args.seed, g=g)
     vals, secs, last = [], [], None
     for _ in range(args.steps):
-        last = oracle_sample(w, rho, target_s=per_step, g=g)
+        last = oracle_sample(w, rho, target_s=per_step, seed=args.seed, g=g)
         vals.append(last["value"])
         secs.append(last["seconds"])
     value = statistics.mean(vals)
@@ -620,6 +620,7 @@ def main():
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="grouped-query layout: K and V hold this many heads, each shared by H / kv-heads "
                          "consecutive query heads (default: as many as Q)")
+    ap.add_argument("--seed", type=int, default=0, help="input seed (rank r draws seed + r)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -163,6 +163,17 @@ SA_API sa_status sa_budget_schedule(const float* densities, int n_steps, int n_c
 #define SA_DEFAULT_MIN_SEQ_LEN 8192
 SA_API int sa_sparse_stage_gate(int N, int min_seq_len, int is_self_attention, int has_token_mask, int is_causal);
 
+/* Why the gate above declines [SDN stage paragraph: the stage records why it
+ * declined]: a bit set per failed condition, 0 when the call takes the
+ * sparse path (sa_sparse_stage_gate returns 1 exactly then).  Host only. */
+typedef enum {
+  SA_DECLINE_NOT_SELF_ATTENTION = 1,
+  SA_DECLINE_TOKEN_MASK = 2,
+  SA_DECLINE_CAUSAL = 4,
+  SA_DECLINE_SHORT = 8
+} sa_decline_reason;
+SA_API int sa_sparse_stage_decline(int N, int min_seq_len, int is_self_attention, int has_token_mask, int is_causal);
+
 /*
  * sa_select_blocks [SDN "selector" + "host sync" paragraphs].
  * Per (batch, active head, 64-row query block i):

@@ -13,6 +13,7 @@ fallback path.  Build it with ``python prompt_aware_head_b200/build.py`` (or
 from __future__ import annotations
 
 import ctypes
+import logging
 import os
 from typing import Optional, Sequence, Tuple
 
@@ -64,6 +65,7 @@ _SIGS = {
     "sa_budget": ([_F, _I], _I),
     "sa_budget_schedule": ([_P, _I, _I, _P, _P], _I),
     "sa_sparse_stage_gate": ([_I, _I, _I, _I, _I], _I),
+    "sa_sparse_stage_decline": ([_I, _I, _I, _I, _I], _I),
     "sa_select_blocks": ([_P, _P, _P, _I, _I, _I, _F, _P, _I, _P, _P, _P, _P, _SZ, _P], _I),
     "sa_select_blocks_noalloc": ([_P, _P, _P, _I, _I, _I, _F, _P, _I, _P, _P, _P, _P], _I),
     "sa_pattern_mask": ([_P, ctypes.POINTER(sa_pattern), _I, _I, _F, _P, _I, _P, _P, _P], _I),
@@ -181,11 +183,31 @@ def sa_budget_schedule(densities, n_cand: int) -> Tuple[np.ndarray, np.ndarray]:
     return k, dense.astype(bool)
 
 
+SA_DECLINE_NOT_SELF_ATTENTION, SA_DECLINE_TOKEN_MASK, SA_DECLINE_CAUSAL, SA_DECLINE_SHORT = 1, 2, 4, 8
+_DECLINE_NAMES = ((SA_DECLINE_NOT_SELF_ATTENTION, "not self attention"), (SA_DECLINE_TOKEN_MASK, "token mask"),
+                  (SA_DECLINE_CAUSAL, "causal"), (SA_DECLINE_SHORT, "below the minimum length"))
+_declines_logged = set()
+_log = logging.getLogger("prompt_aware_head_b200")
+
+
+def sa_sparse_stage_decline(N: int, min_seq_len: int = 0, self_attention: bool = True, token_mask: bool = False,
+                            causal: bool = False) -> int:
+    """Bit set of the reasons the sparse stage declines a call (0: it does not)."""
+    return int(_lib.sa_sparse_stage_decline(int(N), int(min_seq_len), int(bool(self_attention)),
+                                            int(bool(token_mask)), int(bool(causal))))
+
+
 def sa_sparse_stage_gate(N: int, min_seq_len: int = 0, self_attention: bool = True, token_mask: bool = False,
                          causal: bool = False) -> bool:
-    """True when a call should take the block-sparse path (host only)."""
-    return bool(_lib.sa_sparse_stage_gate(int(N), int(min_seq_len), int(bool(self_attention)), int(bool(token_mask)),
-                                          int(bool(causal))))
+    """True when a call should take the block-sparse path (host only).  A
+    decline is logged once per (reasons, N), so a setting that cannot act is
+    visible without repeating every call."""
+    why = sa_sparse_stage_decline(N, min_seq_len, self_attention, token_mask, causal)
+    if why and (why, int(N)) not in _declines_logged:
+        _declines_logged.add((why, int(N)))
+        _log.info("sparse attention declined at N=%d: %s", int(N),
+                  ", ".join(name for bit, name in _DECLINE_NAMES if why & bit))
+    return why == 0
 
 
 def sa_workspace_size(B: int, H: int, N: int, d: int) -> int:

@@ -7,6 +7,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "sa_common.cuh"
 #include "sa_internal.h"
 
@@ -120,6 +122,14 @@ sa_status ws_ok(const void* ws, size_t ws_bytes, int B, int H, int N, int d) {
 
 sa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
 
+// An NVTX range around one ABI call (a no-op unless a profiler is attached).
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
+
 }  // namespace
 
 extern "C" {
@@ -171,9 +181,18 @@ sa_status sa_budget_schedule(const float* densities, int n_steps, int n_cand, in
   return SA_OK;
 }
 
-int sa_sparse_stage_gate(int N, int min_seq_len, int is_self_attention, int has_token_mask, int is_causal) {
+int sa_sparse_stage_decline(int N, int min_seq_len, int is_self_attention, int has_token_mask, int is_causal) {
   const int min_len = min_seq_len > 0 ? min_seq_len : SA_DEFAULT_MIN_SEQ_LEN;
-  return (is_self_attention && !has_token_mask && !is_causal && N >= min_len) ? 1 : 0;
+  int why = 0;
+  if (!is_self_attention) why |= SA_DECLINE_NOT_SELF_ATTENTION;
+  if (has_token_mask) why |= SA_DECLINE_TOKEN_MASK;
+  if (is_causal) why |= SA_DECLINE_CAUSAL;
+  if (N < min_len) why |= SA_DECLINE_SHORT;
+  return why;
+}
+
+int sa_sparse_stage_gate(int N, int min_seq_len, int is_self_attention, int has_token_mask, int is_causal) {
+  return sa_sparse_stage_decline(N, min_seq_len, is_self_attention, has_token_mask, is_causal) == 0 ? 1 : 0;
 }
 
 sa_status sa_build_layout(const sa_segment* segs, int nseg, int N, int block, sa_layout** out) {
@@ -312,6 +331,7 @@ static bool kv_heads_ok(int H, int H_kv) { return H_kv >= 1 && H_kv <= H && H % 
 sa_status sa_select_blocks_gqa(const sa_layout* L, const void* Q, const void* K, int B, int H, int H_kv, int d,
                                float density, const uint8_t* head_mask, int min_active, int32_t* idx,
                                int32_t* counts, float* scores_out, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  CallRange range("sa_select_blocks");
   if (!L || !Q || !K || !idx || !counts) return SA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K)) return SA_ERR_INVALID_ARG;
   if (B <= 0 || (d != 64 && d != 128) || !kv_heads_ok(H, H_kv)) return SA_ERR_SHAPE;
@@ -339,6 +359,7 @@ sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void* K, int
 sa_status sa_select_blocks_noalloc_gqa(const sa_layout* L, const void* Q, const void* K, int B, int H, int H_kv,
                                        int d, float density, const uint8_t* head_mask, int min_active, int32_t* idx,
                                        int32_t* counts, float* scores_out, sa_stream_t stream) {
+  CallRange range("sa_select_blocks_noalloc");
   if (!L || !Q || !K || !idx || !counts) return SA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K)) return SA_ERR_INVALID_ARG;
   if (B <= 0 || (d != 64 && d != 128) || !kv_heads_ok(H, H_kv)) return SA_ERR_SHAPE;
@@ -368,6 +389,7 @@ sa_status sa_select_blocks_noalloc(const sa_layout* L, const void* Q, const void
 sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H, float density,
                           const uint8_t* head_mask, int min_active, int32_t* idx, int32_t* counts,
                           sa_stream_t stream) {
+  CallRange range("sa_pattern_mask");
   if (!L || !p || !idx || !counts) return SA_ERR_INVALID_ARG;
   if (B <= 0) return SA_ERR_SHAPE;
   if (p->kind < SA_PAT_RADIAL || p->kind > SA_PAT_DILATED) return SA_ERR_INVALID_ARG;
@@ -400,6 +422,7 @@ static sa_status attention_args_ok(const void* Q, const void* K, const void* V, 
 
 sa_status sa_attention_plan(const int32_t* idx, const int32_t* counts, int B, int H, int N, int d, int cap,
                             const uint8_t* head_mask, int min_active, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  CallRange range("sa_attention_plan");
   if (!idx || !counts) return SA_ERR_INVALID_ARG;
   if (B <= 0 || (d != 64 && d != 128) || N <= 0 || N % kBlock || N / kBlock > kMaxBlocks) return SA_ERR_SHAPE;
   if (cap < 1 || cap > N / kBlock) return SA_ERR_SHAPE;
@@ -418,6 +441,7 @@ sa_status sa_attention_plan(const int32_t* idx, const int32_t* counts, int B, in
 sa_status sa_attention_run_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N, int d,
                                const uint8_t* head_mask, int min_active, float softmax_scale, void* O, void* ws,
                                size_t ws_bytes, sa_stream_t stream) {
+  CallRange range("sa_attention_run");
   sa_status st = attention_args_ok(Q, K, V, O, B, H, H_kv, N, d, &softmax_scale);
   if (st != SA_OK) return st;
   uint64_t bits = 0;
@@ -457,6 +481,7 @@ sa_status sa_block_sparse_attention(const void* Q, const void* K, const void* V,
 
 sa_status sa_dense_attention_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N, int d,
                                  float softmax_scale, void* O, void* ws, size_t ws_bytes, sa_stream_t stream) {
+  CallRange range("sa_dense_attention");
   sa_status st = attention_args_ok(Q, K, V, O, B, H, H_kv, N, d, &softmax_scale);
   if (st != SA_OK) return st;
   if (!ws || !aligned16(ws) || ws_bytes < sizeof(WsHeader)) return SA_ERR_WORKSPACE;

@@ -28,7 +28,7 @@ def _reference_line(*extra):
     return json.loads(lines[0])
 
 
-@pytest.mark.parametrize("extra", [(), ("--kv-heads", "2")])
+@pytest.mark.parametrize("extra", [(), ("--kv-heads", "2"), ("--seed", "9")])
 def test_reference_arm_line(extra):
     d = _reference_line(*extra)
     assert d["impl"] == "reference"
@@ -39,7 +39,7 @@ def test_reference_arm_line(extra):
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert cb["split"]["select_ms_per_head"] > 0 and cb["split"]["attention_us_per_row"] > 0
     assert d["e2e"] == {"value": d["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
-    assert d["config"]["H_kv"] == (2 if extra else 4)
+    assert d["config"]["H_kv"] == (2 if "--kv-heads" in extra else 4)
     assert d["config"]["workload"].startswith("tiny: B1 H4")
 
 

@@ -61,3 +61,28 @@ def test_stage_gate(sa):
     assert not sa.sa_sparse_stage_gate(16896, self_attention=False)
     assert not sa.sa_sparse_stage_gate(16896, token_mask=True)
     assert not sa.sa_sparse_stage_gate(16896, causal=True)
+
+
+def test_decline_reasons(sa):
+    assert sa.sa_sparse_stage_decline(16896) == 0
+    assert sa.sa_sparse_stage_decline(4096) == sa.SA_DECLINE_SHORT
+    assert sa.sa_sparse_stage_decline(16896, self_attention=False, causal=True) == \
+        sa.SA_DECLINE_NOT_SELF_ATTENTION | sa.SA_DECLINE_CAUSAL
+    assert sa.sa_sparse_stage_decline(100, token_mask=True) == sa.SA_DECLINE_TOKEN_MASK | sa.SA_DECLINE_SHORT
+    for N in (100, 8192, 40000):
+        for flags in ((True, False, False), (False, True, True), (True, True, False)):
+            assert sa.sa_sparse_stage_gate(N, 0, *flags) == (sa.sa_sparse_stage_decline(N, 0, *flags) == 0)
+
+
+def test_declines_are_logged_once_per_reason_and_length(sa, caplog):
+    import logging
+    caplog.set_level(logging.INFO, logger="prompt_aware_head_b200")
+    for _ in range(3):
+        assert not sa.sa_sparse_stage_gate(1234)              # short: logged once
+        assert not sa.sa_sparse_stage_gate(1234, causal=True)  # another reason set: once more
+        assert not sa.sa_sparse_stage_gate(1298)              # another length: once more
+        assert sa.sa_sparse_stage_gate(20000)                 # taken: nothing
+    msgs = [r.getMessage() for r in caplog.records if r.name == "prompt_aware_head_b200"]
+    assert msgs == ["sparse attention declined at N=1234: below the minimum length",
+                    "sparse attention declined at N=1234: causal, below the minimum length",
+                    "sparse attention declined at N=1298: below the minimum length"]
