@@ -157,8 +157,11 @@ SA_API sa_status sa_budget_schedule(const float* densities, int n_steps, int n_c
  * default, the sparse/dense crossover measured there), and the absence of a
  * token mask or causal flag, which a block-only mask cannot combine with].
  * Returns 1 when is_self_attention != 0, has_token_mask == 0, is_causal == 0
- * and N >= min_seq_len (min_seq_len <= 0 means SA_DEFAULT_MIN_SEQ_LEN),
- * else 0 (stay dense).  Host only.
+ * and N >= min_seq_len, else 0 (stay dense).  The default floor is passed
+ * explicitly (SA_DEFAULT_MIN_SEQ_LEN); 0 means no floor, so every length
+ * qualifies [SDN: 0 means no floor, the default is stated rather than hidden
+ * behind a sentinel].  Negative values are reserved for a derived floor and
+ * act as the default until one is defined.  Host only.
  */
 #define SA_DEFAULT_MIN_SEQ_LEN 8192
 SA_API int sa_sparse_stage_gate(int N, int min_seq_len, int is_self_attention, int has_token_mask, int is_causal);

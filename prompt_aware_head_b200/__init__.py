@@ -190,15 +190,15 @@ _declines_logged = set()
 _log = logging.getLogger("prompt_aware_head_b200")
 
 
-def sa_sparse_stage_decline(N: int, min_seq_len: int = 0, self_attention: bool = True, token_mask: bool = False,
-                            causal: bool = False) -> int:
+def sa_sparse_stage_decline(N: int, min_seq_len: int = DEFAULT_MIN_SEQ_LEN, self_attention: bool = True,
+                            token_mask: bool = False, causal: bool = False) -> int:
     """Bit set of the reasons the sparse stage declines a call (0: it does not)."""
     return int(_lib.sa_sparse_stage_decline(int(N), int(min_seq_len), int(bool(self_attention)),
                                             int(bool(token_mask)), int(bool(causal))))
 
 
-def sa_sparse_stage_gate(N: int, min_seq_len: int = 0, self_attention: bool = True, token_mask: bool = False,
-                         causal: bool = False) -> bool:
+def sa_sparse_stage_gate(N: int, min_seq_len: int = DEFAULT_MIN_SEQ_LEN, self_attention: bool = True,
+                         token_mask: bool = False, causal: bool = False) -> bool:
     """True when a call should take the block-sparse path (host only).  A
     decline is logged once per (reasons, N), so a setting that cannot act is
     visible without repeating every call."""

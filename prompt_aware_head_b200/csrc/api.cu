@@ -182,7 +182,7 @@ sa_status sa_budget_schedule(const float* densities, int n_steps, int n_cand, in
 }
 
 int sa_sparse_stage_decline(int N, int min_seq_len, int is_self_attention, int has_token_mask, int is_causal) {
-  const int min_len = min_seq_len > 0 ? min_seq_len : SA_DEFAULT_MIN_SEQ_LEN;
+  const int min_len = min_seq_len >= 0 ? min_seq_len : SA_DEFAULT_MIN_SEQ_LEN;  // 0: no floor
   int why = 0;
   if (!is_self_attention) why |= SA_DECLINE_NOT_SELF_ATTENTION;
   if (has_token_mask) why |= SA_DECLINE_TOKEN_MASK;

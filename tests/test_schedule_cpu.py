@@ -58,6 +58,8 @@ def test_stage_gate(sa):
     assert sa.sa_sparse_stage_gate(16896) and sa.sa_sparse_stage_gate(33280)
     assert not sa.sa_sparse_stage_gate(4096)                      # the sdxl shape stays dense by default
     assert sa.sa_sparse_stage_gate(4096, min_seq_len=4096)
+    assert sa.sa_sparse_stage_gate(64, min_seq_len=0)             # 0: no floor, every length qualifies
+    assert not sa.sa_sparse_stage_gate(8191, min_seq_len=-1)      # negative: reserved, the default floor for now
     assert not sa.sa_sparse_stage_gate(16896, self_attention=False)
     assert not sa.sa_sparse_stage_gate(16896, token_mask=True)
     assert not sa.sa_sparse_stage_gate(16896, causal=True)
@@ -70,8 +72,9 @@ def test_decline_reasons(sa):
         sa.SA_DECLINE_NOT_SELF_ATTENTION | sa.SA_DECLINE_CAUSAL
     assert sa.sa_sparse_stage_decline(100, token_mask=True) == sa.SA_DECLINE_TOKEN_MASK | sa.SA_DECLINE_SHORT
     for N in (100, 8192, 40000):
-        for flags in ((True, False, False), (False, True, True), (True, True, False)):
-            assert sa.sa_sparse_stage_gate(N, 0, *flags) == (sa.sa_sparse_stage_decline(N, 0, *flags) == 0)
+        for floor in (0, 8192, -1):
+            for flags in ((True, False, False), (False, True, True), (True, True, False)):
+                assert sa.sa_sparse_stage_gate(N, floor, *flags) == (sa.sa_sparse_stage_decline(N, floor, *flags) == 0)
 
 
 def test_declines_are_logged_once_per_reason_and_length(sa, caplog):
