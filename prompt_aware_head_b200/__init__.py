@@ -39,6 +39,7 @@ SA_PAT_RADIAL, SA_PAT_WINDOW_GLOBAL, SA_PAT_DILATED = range(3)
 # per layer and the default fraction of heads to skip.
 MIN_ACTIVE_HEADS = 4
 DEFAULT_SPARSITY = 0.5
+MAX_QUALITY_LOSS = 0.02  # the crate's quality-loss bound; its gate needs trained models and is not built here
 DEFAULT_MIN_SEQ_LEN = 8192  # SA_DEFAULT_MIN_SEQ_LEN
 
 

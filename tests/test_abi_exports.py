@@ -97,3 +97,11 @@ def test_grouped_head_counts_checked_before_any_launch(lib):
             lib.sa_block_sparse_attention_gqa(fake, fake, fake, 1, 6, H_kv, 512, 64, fake, fake, 8, None, 0, 0.0,
                                               fake, fake, 1 << 30, stream=0)
         assert e.value.status == lib.SA_ERR_SHAPE
+
+
+def test_binding_constants_match_the_crate(lib):
+    from tests.conftest import read_golden
+    g = read_golden("crate_constants.txt")
+    assert lib.MIN_ACTIVE_HEADS == int(g["MIN_ACTIVE_HEADS"])
+    assert lib.DEFAULT_SPARSITY == float(g["DEFAULT_SPARSITY"])
+    assert lib.MAX_QUALITY_LOSS == float(g["MAX_QUALITY_LOSS"])
