@@ -21,6 +21,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -82,6 +83,28 @@ def time_stats(times_ms):
         raise ValueError("no times")
     p90 = xs[max(0, -(-9 * len(xs) // 10) - 1)]
     return {"mean": round(statistics.mean(xs), 5), "median": round(statistics.median(xs), 5), "p90": round(p90, 5)}
+
+
+def crossover(points):
+    """Sparse/dense crossover from [(N, sparse_ms, dense_ms), ...].
+
+    Returns (N*, kind): the smallest length from which the sparse step stays
+    faster than dense, interpolated linearly in log N between the last point
+    where it was not and the next ("interpolated"); the first N when sparse
+    wins at every point ("at or below"); None when it never wins at the
+    largest N ("above")."""
+    pts = sorted(points)
+    if not pts:
+        raise ValueError("no points")
+    r = [d / s for _, s, d in pts]  # speedup of sparse over dense
+    if r[-1] < 1.0:
+        return None, "above"
+    last_loss = max((q for q in range(len(pts)) if r[q] < 1.0), default=None)
+    if last_loss is None:
+        return float(pts[0][0]), "at or below"
+    na, nb = math.log(pts[last_loss][0]), math.log(pts[last_loss + 1][0])
+    ra, rb = r[last_loss], r[last_loss + 1]
+    return float(math.exp(na + (1.0 - ra) / (rb - ra) * (nb - na))), "interpolated"
 
 
 def job_value(flops_per_rank, ms_max, world):
@@ -485,6 +508,72 @@ def run_ours(args):
         print(json.dumps(out), flush=True)
 
 
+def run_crossover(args):
+    """Sparse step (select + plan + attention) against this library's dense
+    kernel over sequence lengths, on one GPU: the joint config's heads and
+    head size at its density, image tokens only (rows of 128 tokens)."""
+    import torch
+    import prompt_aware_head_b200 as sa
+    from workloads import make_workload
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--crossover runs on one GPU")
+    dev = torch.device("cuda", 0)
+    base = WORKLOADS["joint"]
+    rho = args.density if args.density else base.densities[0]
+    stream = torch.cuda.current_stream(dev)
+    scratch = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    points = []
+    for N in (2048, 4096, 6144, 8192, 12288, 16384, 24576, 32768):
+        w = make_workload("joint", N=N, segments=(), grid=(N // 128, 128))
+        B, H, d = w.B, w.H, w.d
+        Q, K, V = (torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16) for x in make_qkv(w))
+        L = sa.Layout([], N)
+        ws_bytes = sa.sa_workspace_size(B, H, N, d)
+        ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+        sa.sa_workspace_init(ws, ws_bytes, stream)
+        idx = torch.zeros((B, H, w.nB, L.cap), dtype=torch.int32, device=dev)
+        counts = torch.zeros((B, H, w.nB), dtype=torch.int32, device=dev)
+        O = torch.empty_like(Q)
+
+        def sparse():
+            sa.sa_select_blocks(L, Q, K, B, H, d, rho, None, 0, idx, counts, None, ws, ws_bytes, stream)
+            sa.sa_block_sparse_attention(Q, K, V, B, H, N, d, idx, counts, L.cap, None, 0, 0.0, O, ws, ws_bytes,
+                                         stream)
+
+        def dense():
+            sa.sa_dense_attention(Q, K, V, B, H, N, d, 0.0, O, ws, ws_bytes, stream)
+
+        ms = []
+        for fn in (sparse, dense):
+            for _ in range(args.warmup):
+                fn()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for a, b in ev:
+                scratch.fill_(1.0)  # flush L2 outside the events
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(statistics.mean(a.elapsed_time(b) for a, b in ev))
+        assert sa.sa_check(ws, stream) == sa.SA_OK
+        points.append((N, ms[0], ms[1]))
+        L.release()
+        del Q, K, V, O, ws, idx, counts
+    n_star, kind = crossover(points)
+    print(json.dumps({
+        "metric": "sparse/dense crossover sequence length", "value": round(n_star) if n_star else None,
+        "unit": "tokens", "crossover": kind, "higher_is_better": False, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "dtype": "bf16", "data": "synthetic (seeded)",
+        "config": {"workload": "B1 H24 d128, image tokens only (rows of 128), density %.2f" % rho,
+                   "l2": "flushed before every timed call (512 MB write outside the events)",
+                   "sparse": "sa_select_blocks + sa_block_sparse_attention", "dense": "sa_dense_attention"},
+        "points": [{"N": n, "sparse_ms": round(a, 5), "dense_ms": round(b, 5), "speedup": round(b / a, 3)}
+                   for n, a, b in points],
+    }), flush=True)
+
+
 def run_reference(args):
     """The fp64 CPU oracle as it stands, timed on the host cores (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
@@ -538,10 +627,15 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--crossover", action="store_true",
+                    help="instead of the step benchmark: the sequence length from which the sparse step beats dense "
+                         "(one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.crossover:
+        run_crossover(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
