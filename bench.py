@@ -301,6 +301,9 @@ def run_ours(args):
                                     stream)
         elif args.pattern == "radial":
             sa.sa_pattern_mask(L, sa.SA_PAT_RADIAL, B, H, rho, mask, w.min_active, idx, counts, stream=stream)
+        elif args.pattern == "random":
+            sa.sa_pattern_mask(L, sa.SA_PAT_RANDOM, B, H, rho, mask, w.min_active, idx, counts, stream=stream,
+                               seed=rank)
         else:
             sa.sa_pattern_mask(L, sa.SA_PAT_WINDOW_GLOBAL, B, H, rho, mask, w.min_active, idx, counts,
                                window_tokens=512, n_global_blocks=8, stream=stream)
@@ -614,9 +617,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="joint")
     ap.add_argument("--density", type=float, default=None)
-    ap.add_argument("--pattern", choices=["content", "radial", "window"], default="content",
+    ap.add_argument("--pattern", choices=["content", "radial", "random", "window"], default="content",
                     help="block lists from the content selector (default), or a control pattern at the same pins: "
-                         "radial band at the same k, or a 512-token window + 8 global blocks")
+                         "radial band at the same k, random blocks at the same k, or a 512-token window + 8 global "
+                         "blocks")
     ap.add_argument("--kv-heads", type=int, default=None,
                     help="grouped-query layout: K and V hold this many heads, each shared by H / kv-heads "
                          "consecutive query heads (default: as many as Q)")

@@ -89,8 +89,8 @@ typedef enum { SA_BLOCK_PIN = 0, SA_BLOCK_SPARSE = 1, SA_BLOCK_DROP = 2 } sa_blo
 
 typedef struct sa_layout sa_layout;  /* opaque, library-owned, refcounted, cached */
 
-/* Control patterns [SDN "radial control"; GLO sliding window, dilated, global]. */
-typedef enum { SA_PAT_RADIAL = 0, SA_PAT_WINDOW_GLOBAL = 1, SA_PAT_DILATED = 2 } sa_pattern_kind;
+/* Control patterns [SDN "radial control"; GLO sliding window, dilated, global, random]. */
+typedef enum { SA_PAT_RADIAL = 0, SA_PAT_WINDOW_GLOBAL = 1, SA_PAT_DILATED = 2, SA_PAT_RANDOM = 3 } sa_pattern_kind;
 
 typedef struct {
   int32_t kind;             /* sa_pattern_kind                                        */
@@ -98,6 +98,7 @@ typedef struct {
   int32_t n_global_blocks;  /* G: the first G sparsifiable blocks are global rows and
                                columns (window and dilated patterns)                  */
   int32_t dilation;         /* r: dilated keys satisfy (q - key) % r == 0 (r >= 1)    */
+  uint64_t seed;            /* random pattern: SplitMix64 seed of the draw            */
 } sa_pattern;
 
 /* Optional per-call statistics [HS KernelStats]: filled only by sa_density. */
@@ -238,7 +239,12 @@ SA_API sa_status sa_select_blocks_noalloc(const sa_layout* L, const void* Q, con
  *     columns; those G blocks' rows are dense over non-DROP blocks.
  *   DILATED: SPARSE blocks holding some key with |q - key| <= W and
  *     (q - key) % r == 0 for some query of block i, plus G globals as above.
- * density is used by RADIAL only.  No workspace needed.
+ *   RANDOM: the diagonal and k - 1 = sa_budget(density, C) - 1 other SPARSE
+ *     blocks drawn uniformly without replacement, one draw per row for every
+ *     head: block j of row i ranks by the top 21 bits of output i*nB + j + 1
+ *     of SplitMix64 (Steele, Lea and Flood 2014) seeded with `seed`, larger
+ *     first, ties to the lower j.
+ * density is used by RADIAL and RANDOM only.  No workspace needed.
  */
 SA_API sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H, float density,
                           const uint8_t* head_mask, int min_active,

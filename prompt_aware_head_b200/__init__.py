@@ -33,7 +33,7 @@ SA_OK, SA_ERR_INVALID_ARG, SA_ERR_SHAPE, SA_ERR_LAYOUT, SA_ERR_HEAD_MASK, SA_ERR
     SA_ERR_BAD_INDEX, SA_ERR_TIMEOUT, SA_ERR_UNSUPPORTED, SA_ERR_CUDA = range(10)
 SA_SEG_TEXT, SA_SEG_PAD, SA_SEG_IMAGE, SA_SEG_OTHER = range(4)
 SA_BLOCK_PIN, SA_BLOCK_SPARSE, SA_BLOCK_DROP = range(3)
-SA_PAT_RADIAL, SA_PAT_WINDOW_GLOBAL, SA_PAT_DILATED = range(3)
+SA_PAT_RADIAL, SA_PAT_WINDOW_GLOBAL, SA_PAT_DILATED, SA_PAT_RANDOM = range(4)
 
 # Constants of the haagenti_sparse crate (lib.rs): minimum heads kept active
 # per layer and the default fraction of heads to skip.
@@ -49,7 +49,7 @@ class sa_segment(ctypes.Structure):
 
 class sa_pattern(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("window_tokens", ctypes.c_int32),
-                ("n_global_blocks", ctypes.c_int32), ("dilation", ctypes.c_int32)]
+                ("n_global_blocks", ctypes.c_int32), ("dilation", ctypes.c_int32), ("seed", ctypes.c_uint64)]
 
 
 class sa_stats(ctypes.Structure):
@@ -246,8 +246,8 @@ def sa_select_blocks_noalloc(L: Layout, Q, K, B: int, H: int, d: int, density: f
 
 def sa_pattern_mask(L: Layout, kind: int, B: int, H: int, density: float = 1.0, head_mask=None,
                     min_active: int = 0, idx=None, counts=None, window_tokens: int = 0, n_global_blocks: int = 0,
-                    dilation: int = 1, stream=None) -> None:
-    p = sa_pattern(kind, window_tokens, n_global_blocks, dilation)
+                    dilation: int = 1, stream=None, seed: int = 0) -> None:
+    p = sa_pattern(kind, window_tokens, n_global_blocks, dilation, seed)
     mptr, _keep = _host_mask(head_mask)
     _check(_lib.sa_pattern_mask(L.handle, ctypes.byref(p), B, H, ctypes.c_float(density), mptr, min_active,
                                 _addr(idx), _addr(counts), _stream(stream)), "sa_pattern_mask")

@@ -392,9 +392,10 @@ sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H,
   CallRange range("sa_pattern_mask");
   if (!L || !p || !idx || !counts) return SA_ERR_INVALID_ARG;
   if (B <= 0) return SA_ERR_SHAPE;
-  if (p->kind < SA_PAT_RADIAL || p->kind > SA_PAT_DILATED) return SA_ERR_INVALID_ARG;
-  if (p->kind == SA_PAT_RADIAL && !density_ok(density)) return SA_ERR_INVALID_ARG;
-  if (p->kind != SA_PAT_RADIAL && (p->window_tokens < 0 || p->n_global_blocks < 0)) return SA_ERR_INVALID_ARG;
+  if (p->kind < SA_PAT_RADIAL || p->kind > SA_PAT_RANDOM) return SA_ERR_INVALID_ARG;
+  const bool budgeted = p->kind == SA_PAT_RADIAL || p->kind == SA_PAT_RANDOM;  // k from the density
+  if (budgeted && !density_ok(density)) return SA_ERR_INVALID_ARG;
+  if (!budgeted && (p->window_tokens < 0 || p->n_global_blocks < 0)) return SA_ERR_INVALID_ARG;
   if (p->kind == SA_PAT_DILATED && p->dilation < 1) return SA_ERR_INVALID_ARG;
   uint64_t bits = 0;
   sa_status st = head_bits_of(head_mask, H, min_active, &bits);
@@ -402,10 +403,11 @@ sa_status sa_pattern_mask(const sa_layout* L, const sa_pattern* p, int B, int H,
   DeviceInfo di;
   if ((st = check_device(&di)) != SA_OK) return st;
   if (di.id != L->device) return SA_ERR_INVALID_ARG;
-  const int k = p->kind == SA_PAT_RADIAL ? sa_budget(density, L->n_cand) : 0;
-  return from_cuda(launch_pattern(L, p->kind, p->window_tokens, p->n_global_blocks,
+  const int k = budgeted ? sa_budget(density, L->n_cand) : 0;
+  const int kind = p->kind == SA_PAT_RANDOM ? 4 : p->kind;  // the kernel's kind 3 is the dense lists
+  return from_cuda(launch_pattern(L, kind, budgeted ? 0 : p->window_tokens, budgeted ? 0 : p->n_global_blocks,
                                   p->kind == SA_PAT_DILATED ? p->dilation : 1, k, B, H, bits, idx, counts,
-                                  reinterpret_cast<cudaStream_t>(stream)));
+                                  reinterpret_cast<cudaStream_t>(stream), p->seed));
 }
 
 static sa_status attention_args_ok(const void* Q, const void* K, const void* V, const void* O, int B, int H,

@@ -68,9 +68,9 @@ size_t select_noalloc_limit();
 cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int Hkv, int d,
                                   int k, uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out,
                                   cudaStream_t s);
-// kind: 0 radial, 1 window+global, 2 dilated, 3 dense (every non-drop block).
+// kind: 0 radial, 1 window+global, 2 dilated, 3 dense (every non-drop block), 4 random (seed).
 cudaError_t launch_pattern(const sa_layout* L, int kind, int W, int G, int r, int k, int B, int H,
-                           uint64_t head_bits, int32_t* idx, int32_t* counts, cudaStream_t s);
+                           uint64_t head_bits, int32_t* idx, int32_t* counts, cudaStream_t s, uint64_t seed = 0);
 cudaError_t launch_density(const int32_t* counts, int B, int H, int nB, uint64_t head_bits, void* ws,
                            unsigned long long* host_tiles, cudaStream_t s);
 

@@ -702,18 +702,30 @@ __device__ __forceinline__ bool dilated_cover(int i, int j, int W, int r) {
   return first <= hi;
 }
 
+// Output n >= 1 of SplitMix64 (Steele, Lea and Flood 2014) seeded with
+// `seed`: the state advances by the odd constant 0x9E3779B97F4A7C15 per
+// output and is put through the mix (xor-shift 30, multiply, xor-shift 27,
+// multiply, xor-shift 31).  Counter-based: any output is computed directly.
+__device__ __forceinline__ unsigned long long splitmix64_nth(unsigned long long seed, unsigned long long n) {
+  unsigned long long z = seed + n * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// kind: 0 radial, 1 window + global, 2 dilated, 3 dense, 4 random (seed).
 template <int NC>
 __global__ void __launch_bounds__(128) pattern_kernel(const uint8_t* __restrict__ cls,
                                                       const int32_t* __restrict__ sparse_rank, int nB, int kind,
                                                       int W, int G, int r, int k, int BH, int H,
                                                       uint64_t head_bits, int cap, int32_t* __restrict__ idx,
-                                                      int32_t* __restrict__ counts) {
+                                                      int32_t* __restrict__ counts, unsigned long long seed) {
   __shared__ int32_t lst[4][NC * 32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * 4 + w;
   if (i >= nB) return;
   const uint8_t ci = cls[i];
-  const bool row_global = ci == kSparse && kind != 0 && kind != 3 && sparse_rank[i] < G;
+  const bool row_global = ci == kSparse && (kind == 1 || kind == 2) && sparse_rank[i] < G;
   uint32_t keep = 0;
   if (ci == kPin || (ci == kSparse && (kind == 3 || row_global))) {
 #pragma unroll
@@ -735,6 +747,13 @@ __global__ void __launch_bounds__(128) pattern_kernel(const uint8_t* __restrict_
       if (kind == 0) {
         key[c] = ~((static_cast<uint32_t>(abs(i - j)) << 16) | static_cast<uint32_t>(j));
         cand |= 1u << c;
+      } else if (kind == 4) {
+        // the diagonal above every draw; a draw's 21 bits above 1023 - j (nB <= 1024): distinct keys,
+        // larger draw first, ties to the lower j
+        const unsigned long long u =
+            splitmix64_nth(seed, static_cast<unsigned long long>(i) * static_cast<unsigned long long>(nB) + j + 1);
+        key[c] = (j == i) ? 0xFFFFFFFFu : ((static_cast<uint32_t>(u >> 43) << 10) | static_cast<uint32_t>(1023 - j));
+        cand |= 1u << c;
       } else {
         const bool glob = sparse_rank[j] < G;
         const bool cover = (kind == 1) ? window_cover(i, j, W) : dilated_cover(i, j, W, r);
@@ -742,7 +761,7 @@ __global__ void __launch_bounds__(128) pattern_kernel(const uint8_t* __restrict_
       }
     }
     keep = pin | win;
-    if (kind == 0) keep |= warp_topk<NC>(key, cand, k);
+    if (kind == 0 || kind == 4) keep |= warp_topk<NC>(key, cand, k);
   }
   const int n = warp_emit<NC>(keep, lst[w]);
   __syncwarp();
@@ -972,22 +991,22 @@ cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void*
 
 template <int NC>
 static void launch_pattern_t(const sa_layout* L, int kind, int W, int G, int r, int k, int BH, int H,
-                             uint64_t head_bits, int32_t* idx, int32_t* counts, cudaStream_t s) {
+                             uint64_t head_bits, int32_t* idx, int32_t* counts, uint64_t seed, cudaStream_t s) {
   pattern_kernel<NC><<<(L->nB + 3) / 4, 128, 0, s>>>(L->d_cls, L->d_sparse_rank, L->nB, kind, W, G, r, k, BH, H,
-                                                     head_bits, L->cap, idx, counts);
+                                                     head_bits, L->cap, idx, counts, seed);
 }
 
 cudaError_t launch_pattern(const sa_layout* L, int kind, int W, int G, int r, int k, int B, int H,
-                           uint64_t head_bits, int32_t* idx, int32_t* counts, cudaStream_t s) {
+                           uint64_t head_bits, int32_t* idx, int32_t* counts, cudaStream_t s, uint64_t seed) {
   const int BH = B * H;
   switch (chunks_for(L->nB)) {
-    case 2: launch_pattern_t<2>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, s); break;
-    case 4: launch_pattern_t<4>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, s); break;
-    case 8: launch_pattern_t<8>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, s); break;
-    case 12: launch_pattern_t<12>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, s); break;
-    case 17: launch_pattern_t<17>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, s); break;
-    case 24: launch_pattern_t<24>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, s); break;
-    case 32: launch_pattern_t<32>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, s); break;
+    case 2: launch_pattern_t<2>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, seed, s); break;
+    case 4: launch_pattern_t<4>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, seed, s); break;
+    case 8: launch_pattern_t<8>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, seed, s); break;
+    case 12: launch_pattern_t<12>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, seed, s); break;
+    case 17: launch_pattern_t<17>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, seed, s); break;
+    case 24: launch_pattern_t<24>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, seed, s); break;
+    case 32: launch_pattern_t<32>(L, kind, W, G, r, k, BH, H, head_bits, idx, counts, seed, s); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
