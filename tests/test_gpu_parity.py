@@ -171,21 +171,6 @@ def test_pattern_parity(sa, name, kind, W, G, r):
     compare_lists(*buf.lists(), ref_idx, ref_cnt)
 
 
-@pytest.mark.parametrize("name,seed", [("tiny", 0), ("sdxl", 1), ("joint", 2), ("video", 3), ("video", 2 ** 63 + 5)])
-def test_random_pattern_parity(sa, name, seed):
-    # SplitMix64 draws on both sides: the lists must be identical
-    w = WORKLOADS[name]
-    rho = w.densities[0]
-    mask = head_mask_for_layer(w)
-    L = sa.Layout(list(w.segments), w.N)
-    buf = Buffers(sa, w.B, w.H, w.N, w.d, L.cap)
-    sa.sa_pattern_mask(L, sa.SA_PAT_RANDOM, w.B, w.H, rho, mask, w.min_active, buf.idx, buf.counts, seed=seed)
-    cls = oracle.layout(list(w.segments), w.N)
-    ref_idx, ref_cnt = oracle.pattern(cls, oracle.PAT_RANDOM, w.B * w.H, w.H, density=rho, head_mask=mask,
-                                      cap=L.cap, seed=seed)
-    compare_lists(*buf.lists(), ref_idx, ref_cnt)
-
-
 # ------------------------------------------------------------------ attention
 
 def _attention(sa, w, Q, K, V, buf, mask, min_active):
