@@ -2,11 +2,11 @@
 
 Sorts last among the GPU tests.
 
-This size runs the 32-chunk rank kernel, 8 row tiles of the score kernel,
-union lists of up to 1024 entries and 301 MB of union-list workspace.  The
-selection must match the oracle as everywhere else; attention is checked on
-sampled rows and on every row of the pinned text block.  One block more is
-refused before any launch.
+This size runs the 32-chunk rank kernel, 8 row tiles of the score kernel
+and union lists of up to 1024 entries (25 MB of union-list workspace for
+its two heads; 301 MB at 24 heads).  The selection must match the oracle
+as everywhere else; attention is checked on sampled rows and on every row
+of the pinned text block.  One block more is refused before any launch.
 """
 import numpy as np
 import pytest
