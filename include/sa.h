@@ -301,6 +301,28 @@ SA_API sa_status sa_dense_attention_gqa(const void* Q, const void* K, const void
                                         sa_stream_t stream);
 
 /*
+ * Token-level key mask inside the kept tiles [SDN "masked_block": a backend
+ * takes the attention mask and the block mask together].  key_mask is a
+ * device byte array [B][N], 16-byte aligned, nonzero where key n of batch b
+ * may be attended (a padding mask), or NULL for none.  Query row q of block
+ * i attends to key n only when n's block is in idx[b][h][i][0 .. counts) and
+ * key_mask[b][n] != 0; a row left with no key gets O = 0.  The mask is packed
+ * into one 64-bit word per (batch, key block) in the workspace (one small
+ * kernel), and the attention kernel applies it only to kept tiles whose word
+ * is neither all ones nor zero (a zero word skips the tile).  Other arguments
+ * as in the _gqa forms (H_kv = H for plain multi-head attention).
+ */
+SA_API sa_status sa_block_sparse_attention_masked(const void* Q, const void* K, const void* V, int B, int H,
+                                                  int H_kv, int N, int d, const int32_t* idx, const int32_t* counts,
+                                                  int cap, const uint8_t* key_mask, const uint8_t* head_mask,
+                                                  int min_active, float softmax_scale, void* O, void* ws,
+                                                  size_t ws_bytes, sa_stream_t stream);
+SA_API sa_status sa_attention_run_masked(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N,
+                                         int d, const uint8_t* key_mask, const uint8_t* head_mask, int min_active,
+                                         float softmax_scale, void* O, void* ws, size_t ws_bytes,
+                                         sa_stream_t stream);
+
+/*
  * sa_density [SDN "host sync": density is read back only when something
  * asks].  The only call that reads device memory back: it synchronises
  * `stream`.  Any of the outputs may be NULL.

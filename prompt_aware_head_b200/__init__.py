@@ -76,6 +76,9 @@ _SIGS = {
     "sa_block_sparse_attention_gqa": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _F, _P, _P, _SZ, _P], _I),
     "sa_attention_run_gqa": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _F, _P, _P, _SZ, _P], _I),
     "sa_dense_attention_gqa": ([_P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _SZ, _P], _I),
+    "sa_block_sparse_attention_masked": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _F, _P, _P, _SZ, _P],
+                                         _I),
+    "sa_attention_run_masked": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _SZ, _P], _I),
     "sa_density": ([_P, _I, _I, _I, _P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
                     ctypes.POINTER(sa_stats), _P, _SZ, _P], _I),
     "sa_workspace_size": ([_I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
@@ -299,6 +302,26 @@ def sa_dense_attention_gqa(Q, K, V, B: int, H: int, H_kv: int, N: int, d: int, s
     _check(_lib.sa_dense_attention_gqa(_addr(Q), _addr(K), _addr(V), B, H, H_kv, N, d,
                                        ctypes.c_float(softmax_scale), _addr(O), _addr(ws), ws_bytes,
                                        _stream(stream)), "sa_dense_attention_gqa")
+
+
+# Token-level key mask inside the kept tiles: key_mask is a device uint8 [B, N] (nonzero = may be attended).
+
+def sa_block_sparse_attention_masked(Q, K, V, B: int, H: int, H_kv: int, N: int, d: int, idx, counts, cap: int,
+                                     key_mask, head_mask, min_active: int, softmax_scale: float, O, ws, ws_bytes: int,
+                                     stream=None) -> None:
+    mptr, _keep = _host_mask(head_mask)
+    _check(_lib.sa_block_sparse_attention_masked(_addr(Q), _addr(K), _addr(V), B, H, H_kv, N, d, _addr(idx),
+                                                 _addr(counts), cap, _addr(key_mask), mptr, min_active,
+                                                 ctypes.c_float(softmax_scale), _addr(O), _addr(ws), ws_bytes,
+                                                 _stream(stream)), "sa_block_sparse_attention_masked")
+
+
+def sa_attention_run_masked(Q, K, V, B: int, H: int, H_kv: int, N: int, d: int, key_mask, head_mask,
+                            min_active: int, softmax_scale: float, O, ws, ws_bytes: int, stream=None) -> None:
+    mptr, _keep = _host_mask(head_mask)
+    _check(_lib.sa_attention_run_masked(_addr(Q), _addr(K), _addr(V), B, H, H_kv, N, d, _addr(key_mask), mptr,
+                                        min_active, ctypes.c_float(softmax_scale), _addr(O), _addr(ws), ws_bytes,
+                                        _stream(stream)), "sa_attention_run_masked")
 
 
 def sa_density(counts, B: int, H: int, nB: int, head_mask, ws, ws_bytes: int, stream=None):
