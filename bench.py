@@ -21,6 +21,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -84,6 +85,28 @@ def time_stats(times_ms):
     return {"mean": round(statistics.mean(xs), 5), "median": round(statistics.median(xs), 5), "p90": round(p90, 5)}
 
 
+def crossover(points):
+    """Sparse/dense crossover from [(N, sparse_ms, dense_ms), ...].
+
+    Returns (N*, kind): the smallest length from which the sparse step stays
+    faster than dense, interpolated linearly in log N between the last point
+    where it was not and the next ("interpolated"); the first N when sparse
+    wins at every point ("at or below"); None when it never wins at the
+    largest N ("above")."""
+    pts = sorted(points)
+    if not pts:
+        raise ValueError("no points")
+    r = [d / s for _, s, d in pts]  # speedup of sparse over dense
+    if r[-1] < 1.0:
+        return None, "above"
+    last_loss = max((q for q in range(len(pts)) if r[q] < 1.0), default=None)
+    if last_loss is None:
+        return float(pts[0][0]), "at or below"
+    na, nb = math.log(pts[last_loss][0]), math.log(pts[last_loss + 1][0])
+    ra, rb = r[last_loss], r[last_loss + 1]
+    return float(math.exp(na + (1.0 - ra) / (rb - ra) * (nb - na))), "interpolated"
+
+
 def job_value(flops_per_rank, ms_max, world):
     """Whole-job effective TFLOP/s: every rank's flops over the slowest rank's
     time (each rank runs its own batch: weak scaling)."""
@@ -102,6 +125,7 @@ def oracle_sample(w, rho, target_s=10.0, seed=0, g=1):
     cls = oracle.layout(list(w.segments), w.N)
     flops = 0.0
     t_total = 0.0
+    sel_s, att_s = 0.0, 0.0  # unscaled: every timed selection, every timed attention row
     done_heads, done_rows = 0, 0
     for h in heads:
         Q, K, V = make_qkv(w, seed=seed, heads=[h])
@@ -124,6 +148,8 @@ def oracle_sample(w, rho, target_s=10.0, seed=0, g=1):
         t = time.perf_counter()
         oracle.attention(Q, K, V, 1, idx, cnt, rows=rows)
         t_att = time.perf_counter() - t
+        sel_s += t_sel
+        att_s += t_att
         flops += float(np.sum(4.0 * w.d * 64 * cnt[0, rows // 64]))
         t_total += t_att + t_sel * len(rows) / w.N
         done_heads += 1
@@ -138,6 +164,8 @@ def oracle_sample(w, rho, target_s=10.0, seed=0, g=1):
         "kind": "oracle",
         "sample": "%d of %d heads of the workload: fp64 selection per head (charged pro rata to the rows run) + "
                   "fp64 attention for %d query rows in all (%.1f s)" % (done_heads, len(heads), done_rows, t_total),
+        "split": {"select_ms_per_head": round(1e3 * sel_s / max(done_heads, 1), 3),
+                  "attention_us_per_row": round(1e6 * att_s / max(done_rows, 1), 3)},
         "seconds": t_total,
     }
 
@@ -477,6 +505,72 @@ def run_ours(args):
         print(json.dumps(out), flush=True)
 
 
+def run_crossover(args):
+    """Sparse step (select + plan + attention) against this library's dense
+    kernel over sequence lengths, on one GPU: the joint config's heads and
+    head size at its density, image tokens only (rows of 128 tokens)."""
+    import torch
+    import prompt_aware_head_b200 as sa
+    from workloads import make_workload
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--crossover runs on one GPU")
+    dev = torch.device("cuda", 0)
+    base = WORKLOADS["joint"]
+    rho = args.density if args.density else base.densities[0]
+    stream = torch.cuda.current_stream(dev)
+    scratch = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    points = []
+    for N in (2048, 4096, 6144, 8192, 12288, 16384, 24576, 32768):
+        w = make_workload("joint", N=N, segments=(), grid=(N // 128, 128))
+        B, H, d = w.B, w.H, w.d
+        Q, K, V = (torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16) for x in make_qkv(w))
+        L = sa.Layout([], N)
+        ws_bytes = sa.sa_workspace_size(B, H, N, d)
+        ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+        sa.sa_workspace_init(ws, ws_bytes, stream)
+        idx = torch.zeros((B, H, w.nB, L.cap), dtype=torch.int32, device=dev)
+        counts = torch.zeros((B, H, w.nB), dtype=torch.int32, device=dev)
+        O = torch.empty_like(Q)
+
+        def sparse():
+            sa.sa_select_blocks(L, Q, K, B, H, d, rho, None, 0, idx, counts, None, ws, ws_bytes, stream)
+            sa.sa_block_sparse_attention(Q, K, V, B, H, N, d, idx, counts, L.cap, None, 0, 0.0, O, ws, ws_bytes,
+                                         stream)
+
+        def dense():
+            sa.sa_dense_attention(Q, K, V, B, H, N, d, 0.0, O, ws, ws_bytes, stream)
+
+        ms = []
+        for fn in (sparse, dense):
+            for _ in range(args.warmup):
+                fn()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for a, b in ev:
+                scratch.fill_(1.0)  # flush L2 outside the events
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(statistics.mean(a.elapsed_time(b) for a, b in ev))
+        assert sa.sa_check(ws, stream) == sa.SA_OK
+        points.append((N, ms[0], ms[1]))
+        L.release()
+        del Q, K, V, O, ws, idx, counts
+    n_star, kind = crossover(points)
+    print(json.dumps({
+        "metric": "sparse/dense crossover sequence length", "value": round(n_star) if n_star else None,
+        "unit": "tokens", "crossover": kind, "higher_is_better": False, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "dtype": "bf16", "data": "synthetic (seeded)",
+        "config": {"workload": "B1 H24 d128, image tokens only (rows of 128), density %.2f" % rho,
+                   "l2": "flushed before every timed call (512 MB write outside the events)",
+                   "sparse": "sa_select_blocks + sa_block_sparse_attention", "dense": "sa_dense_attention"},
+        "points": [{"N": n, "sparse_ms": round(a, 5), "dense_ms": round(b, 5), "speedup": round(b / a, 3)}
+                   for n, a, b in points],
+    }), flush=True)
+
+
 def run_reference(args):
     """The fp64 CPU oracle as it stands, timed on the host cores (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
@@ -506,7 +600,7 @@ def run_reference(args):
         "config": {"workload": describe(w, rho, H_kv), "B": w.B, "H": w.H, "H_kv": H_kv, "N": w.N, "d": w.d,
                    "density_budget": rho},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last["cores"], "kind": "oracle",
-                         "sample": last["sample"]},
+                         "sample": last["sample"], "split": last["split"]},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
@@ -529,10 +623,15 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--crossover", action="store_true",
+                    help="instead of the step benchmark: the sequence length from which the sparse step beats dense "
+                         "(one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.crossover:
+        run_crossover(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -23,7 +23,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 PIN, SPARSE, DROP = 0, 1, 2
-PAT_RADIAL, PAT_WINDOW_GLOBAL, PAT_DILATED = 0, 1, 2
+PAT_RADIAL, PAT_WINDOW_GLOBAL, PAT_DILATED, PAT_RANDOM = 0, 1, 2, 3
 
 
 def build_oracle(force: bool = False) -> str:
@@ -49,7 +49,7 @@ def _load():
         _lib.oracle_budget.argtypes = [f, i]
         _lib.oracle_budget.restype = i
         _lib.oracle_select.argtypes = [P, P, i, i, i, f, P, i, P, P]
-        _lib.oracle_pattern.argtypes = [P, i, i, i, i, i, i, f, i, i, P, i, P, P]
+        _lib.oracle_pattern.argtypes = [P, i, i, i, i, i, i, f, i, i, P, i, P, P, ctypes.c_uint64]
         _lib.oracle_pattern.restype = i
         _lib.oracle_attention.argtypes = [P, P, P, i, i, i, i, i, i, P, P, i, P, P, dbl, P, ctypes.c_int64, P]
         _lib.oracle_density.argtypes = [P, i, i, i, P, P, P]
@@ -137,8 +137,9 @@ def select(sc: np.ndarray, cls: np.ndarray, H: int, density: float,
 
 def pattern(cls: np.ndarray, kind: int, BH: int, H: int, window: int = 0, n_global: int = 0,
             dilation: int = 1, density: float = 1.0, head_mask: Optional[np.ndarray] = None,
-            cap: Optional[int] = None, block: int = 64):
-    """Radial / window+global / dilated block lists at the layout's pins and drops."""
+            cap: Optional[int] = None, block: int = 64, seed: int = 0):
+    """Radial / window+global / dilated / random block lists at the layout's pins and drops
+    (seed: the random pattern's SplitMix64 seed)."""
     lib = _load()
     nB = cls.shape[0]
     cap = cap_of(cls) if cap is None else cap
@@ -147,7 +148,7 @@ def pattern(cls: np.ndarray, kind: int, BH: int, H: int, window: int = 0, n_glob
     idx = np.full((BH, nB, max(cap, 1)), -1, dtype=np.int32)
     counts = np.zeros((BH, nB), dtype=np.int32)
     rc = lib.oracle_pattern(_ptr(cls), nB, block, kind, window, n_global, dilation, ctypes.c_float(density),
-                            BH, H, _ptr(hm), max(cap, 1), _ptr(idx), _ptr(counts))
+                            BH, H, _ptr(hm), max(cap, 1), _ptr(idx), _ptr(counts), ctypes.c_uint64(seed))
     if rc != 0:
         raise ValueError("bad pattern")
     return idx, counts

@@ -41,7 +41,7 @@
 
 enum { OR_SEG_TEXT = 0, OR_SEG_PAD = 1, OR_SEG_IMAGE = 2, OR_SEG_OTHER = 3 };
 enum { OR_PIN = 0, OR_SPARSE = 1, OR_DROP = 2 };
-enum { OR_PAT_RADIAL = 0, OR_PAT_WINDOW_GLOBAL = 1, OR_PAT_DILATED = 2 };
+enum { OR_PAT_RADIAL = 0, OR_PAT_WINDOW_GLOBAL = 1, OR_PAT_DILATED = 2, OR_PAT_RANDOM = 3 };
 
 static double bf16_to_double(uint16_t b) {
   uint32_t u = (uint32_t)b << 16;
@@ -243,16 +243,31 @@ static int dilated_cover(int i, int j, int block, int W, int r) {
  * columns.  kind 2 DILATED: block cover of {key : |q - key| <= W,
  * (q - key) % r == 0}, plus G globals when G > 0.
  */
+/*
+ * SplitMix64 (Steele, Lea and Flood, "Fast splittable pseudorandom number
+ * generators", OOPSLA 2014): output number n >= 1 of the generator seeded
+ * with `seed`.  The state advances by the odd constant 0x9E3779B97F4A7C15 per
+ * output; an output is the state after its advance, put through the mix
+ * (xor-shift 30, multiply, xor-shift 27, multiply, xor-shift 31).
+ */
+static uint64_t splitmix64_nth(uint64_t seed, uint64_t n) {
+  uint64_t z = seed + n * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
 int oracle_pattern(const uint8_t* cls, int nB, int block, int kind, int W, int G, int r, float density,
-                   int BH, int H, const uint8_t* head_mask, int cap, int32_t* idx, int32_t* counts) {
-  if (kind < 0 || kind > 2) return -1;
+                   int BH, int H, const uint8_t* head_mask, int cap, int32_t* idx, int32_t* counts,
+                   uint64_t seed) {
+  if (kind < 0 || kind > 3) return -1;
   if (kind == OR_PAT_DILATED && r <= 0) return -1;
   int C = 0;
   for (int j = 0; j < nB; ++j) C += (cls[j] == OR_SPARSE);
   int k = oracle_budget(density, C);
   uint8_t* global = (uint8_t*)calloc((size_t)nB, 1);
   int g = 0;
-  for (int j = 0; j < nB && g < G && kind != OR_PAT_RADIAL; ++j)
+  for (int j = 0; j < nB && g < G && kind != OR_PAT_RADIAL && kind != OR_PAT_RANDOM; ++j)
     if (cls[j] == OR_SPARSE) { global[j] = 1; ++g; }
   uint8_t* keep = (uint8_t*)malloc((size_t)nB);
   cand_t* cand = (cand_t*)malloc(sizeof(cand_t) * (size_t)(nB > 0 ? nB : 1));
@@ -267,6 +282,21 @@ int oracle_pattern(const uint8_t* cls, int nB, int block, int kind, int W, int G
           for (int j = 0; j < nB; ++j) {
             if (cls[j] != OR_SPARSE) continue;
             cand[nc].key = -(double)abs(i - j);   /* nearer first */
+            cand[nc].j = j;
+            ++nc;
+          }
+          qsort(cand, (size_t)nc, sizeof(cand_t), cand_cmp);
+          for (int q = 0; q < k && q < nc; ++q) keep[cand[q].j] = 1;
+        } else if (kind == OR_PAT_RANDOM) {
+          /* [GLO random: each query attends to a fixed set of keys sampled
+           * uniformly at random]: the diagonal, then the k - 1 other sparse
+           * blocks ranked by the top 21 bits of output i*nB + j + 1, larger
+           * first (ties: lower block), the same for every head */
+          int nc = 0;
+          for (int j = 0; j < nB; ++j) {
+            if (cls[j] != OR_SPARSE) continue;
+            cand[nc].key = (j == i) ? INFINITY
+                                    : (double)(splitmix64_nth(seed, (uint64_t)i * (uint64_t)nB + (uint64_t)j + 1) >> 43);
             cand[nc].j = j;
             ++nc;
           }

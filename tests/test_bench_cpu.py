@@ -37,6 +37,7 @@ def test_reference_arm_line(extra):
     assert d["dtype"] == "f64"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert cb["split"]["select_ms_per_head"] > 0 and cb["split"]["attention_us_per_row"] > 0
     assert d["e2e"] == {"value": d["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["H_kv"] == (2 if extra else 4)
     assert d["config"]["workload"].startswith("tiny: B1 H4")
@@ -88,3 +89,15 @@ def test_time_stats():
     assert bench.time_stats([1, 2, 3])["p90"] == 3.0
     with pytest.raises(ValueError):
         bench.time_stats([])
+
+
+def test_crossover_interpolates_in_log_n():
+    # speedups 0.5 at 4096 and 2.0 at 16384: 1.0 lies a third of the way in log N, at 4096 * 4^(1/3)
+    n, kind = bench.crossover([(4096, 2.0, 1.0), (16384, 1.0, 2.0)])
+    assert kind == "interpolated" and abs(n - 4096 * 4 ** (1 / 3)) < 1e-6
+    # the last loss counts: a win below a later loss is ignored
+    n, kind = bench.crossover([(2048, 1.0, 1.5), (4096, 1.0, 0.9), (8192, 1.0, 1.1)])
+    assert kind == "interpolated" and 4096 < n < 8192
+    assert bench.crossover([(2048, 1.0, 1.2), (4096, 1.0, 3.0)]) == (2048.0, "at or below")
+    assert bench.crossover([(2048, 2.0, 1.0), (4096, 2.0, 1.5)]) == (None, "above")
+    assert bench.crossover([(8192, 1.0, 1.0)]) == (8192.0, "at or below")  # equal times count as a win

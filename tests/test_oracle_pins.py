@@ -454,3 +454,45 @@ def test_key_mask_closed_forms():
     one_cnt = np.ones((B * H, w.nB), np.int32)
     out = oracle.attention(_bits(np.ones((B, H, N, w.d))), K, V, H, one_idx, one_cnt, key_mask=km)
     assert np.all(out == 0)
+
+
+# ---------------------------------------------------------------- random-block control pattern
+
+@pytest.mark.parametrize("name", ["tiny", "joint"])
+def test_random_pattern_invariants(name):
+    w = WORKLOADS[name]
+    cls = oracle.layout(list(w.segments), w.N)
+    rho = w.densities[0]
+    C, P = int(np.sum(cls == oracle.SPARSE)), int(np.sum(cls == oracle.PIN))
+    k = oracle.budget(rho, C)
+    idx, counts = oracle.pattern(cls, oracle.PAT_RANDOM, 1, 1, density=rho, seed=7)
+    pins = set(np.flatnonzero(cls == oracle.PIN).tolist())
+    for i in range(w.nB):
+        row = idx[0, i, :counts[0, i]].tolist()
+        if cls[i] == oracle.DROP:
+            assert counts[0, i] == 0
+        elif cls[i] == oracle.PIN:
+            assert row == np.flatnonzero(cls != oracle.DROP).tolist()
+        else:
+            assert len(row) == P + k and i in row and pins <= set(row)
+            assert all(cls[j] != oracle.DROP for j in row) and row == sorted(set(row))
+    again, _ = oracle.pattern(cls, oracle.PAT_RANDOM, 1, 1, density=rho, seed=7)
+    other, _ = oracle.pattern(cls, oracle.PAT_RANDOM, 1, 1, density=rho, seed=8)
+    assert np.array_equal(again, idx) and not np.array_equal(other, idx)
+
+
+def test_random_pattern_draws_uniform_subsets():
+    # 6 sparsifiable blocks, k = 3: the diagonal plus 2 of the other 5, each of the 10 pairs equally likely
+    cls = np.full(6, oracle.SPARSE, np.uint8)
+    n = 20000
+    for i in (0, 3):
+        tally = {}
+        for seed in range(n):
+            idx, counts = oracle.pattern(cls, oracle.PAT_RANDOM, 1, 1, density=0.5, seed=seed)
+            row = idx[0, i, :counts[0, i]].tolist()
+            assert len(row) == 3 and i in row
+            key = tuple(j for j in row if j != i)
+            tally[key] = tally.get(key, 0) + 1
+        assert len(tally) == 10
+        # each count is Binomial(20000, 0.1): mean 2000, sd 42.4; 250 is about 6 sd
+        assert all(abs(c - n / 10) < 250 for c in tally.values()), tally
