@@ -32,7 +32,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import WORKLOADS, head_mask_for_layer, make_qkv  # noqa: E402
+from workloads import SEG_PAD, WORKLOADS, head_mask_for_layer, make_qkv  # noqa: E402
 
 METRIC = "effective TFLOP/s of block-sparse attention; speedup vs dense at 30% density"
 UNIT = "TFLOP/s"
@@ -293,6 +293,13 @@ def run_ours(args):
     scratch = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev) if flush else None
     k_budget = sa.sa_budget(rho, L.n_cand)
     dense_short = k_budget >= L.n_cand
+    km_dev = None  # --pad-mask: the layout's padding tokens masked as keys inside kept tiles
+    if args.pad_mask:
+        km = np.ones((B, N), np.uint8)
+        for kind, start, length in w.segments:
+            if kind == SEG_PAD:
+                km[:, start:start + length] = 0
+        km_dev = torch.from_numpy(km).to(dev)
     n_masked = int(H - mask.sum())
 
     def select(q, k):
@@ -317,14 +324,16 @@ def run_ours(args):
         sa.sa_attention_plan(idx, counts, B, H, N, d, L.cap, mask, w.min_active, ws, ws_bytes, stream)
         if ev is not None:
             ev[2].record(stream)
-        sa.sa_attention_run_gqa(Q, K, V, B, H, H_kv, N, d, mask, w.min_active, 0.0, O, ws, ws_bytes, stream)
+        sa.sa_attention_run_masked(Q, K, V, B, H, H_kv, N, d, km_dev, mask, w.min_active, 0.0, O, ws, ws_bytes,
+                                   stream)
         if ev is not None:
             ev[3].record(stream)
 
     # selection (pool, scores, rank; one kernel for a pattern or a budget that
     # covers every candidate), planner (rows, order), attention (+ zeroing of
     # skipped heads)
-    launches_per_step = (1 if dense_short or args.pattern != "content" else 3) + 2 + 1 + (1 if n_masked else 0)
+    launches_per_step = ((1 if dense_short or args.pattern != "content" else 3) + 2 + 1 + (1 if n_masked else 0)
+                         + (1 if km_dev is not None else 0))
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -420,8 +429,8 @@ def run_ours(args):
         if i >= 2:
             stream.wait_event(out_done[i - 2])
         select(q, k)
-        sa.sa_block_sparse_attention_gqa(q, k, v, B, H, H_kv, N, d, idx, counts, L.cap, mask, w.min_active, 0.0, o,
-                                         ws, ws_bytes, stream)
+        sa.sa_block_sparse_attention_masked(q, k, v, B, H, H_kv, N, d, idx, counts, L.cap, km_dev, mask,
+                                            w.min_active, 0.0, o, ws, ws_bytes, stream)
         comp_done[i].record(stream)
         s_out.wait_event(comp_done[i])
         with torch.cuda.stream(s_out):
@@ -459,6 +468,7 @@ def run_ours(args):
         "config": {
             "workload": describe(w, rho, H_kv),
             "B": B, "H": H, "H_kv": H_kv, "N": N, "d": d, "density_budget": rho, "lists": args.pattern,
+            "key_mask": "padding tokens masked inside kept tiles" if km_dev is not None else None,
             "density_realized": round(tiles / (B * n_act * w.nB ** 2), 5),
             "selected_tiles": int(tiles),
             "l2": "flushed between steps (512 MB write outside the per-step events)" if flush
@@ -625,6 +635,8 @@ def main():
                     help="grouped-query layout: K and V hold this many heads, each shared by H / kv-heads "
                          "consecutive query heads (default: as many as Q)")
     ap.add_argument("--seed", type=int, default=0, help="input seed (rank r draws seed + r)")
+    ap.add_argument("--pad-mask", action="store_true",
+                    help="mask the layout's padding tokens as keys inside the kept tiles (token-level key mask)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -155,16 +155,26 @@ SA_API sa_status sa_budget_schedule(const float* densities, int n_steps, int n_c
 /*
  * Whether a call takes the block-sparse path [SDN stage paragraph: the
  * stage gates on self attention, a minimum sequence length (8192 tokens by
- * default, the sparse/dense crossover measured there), and the absence of a
- * token mask or causal flag, which a block-only mask cannot combine with].
- * Returns 1 when is_self_attention != 0, has_token_mask == 0, is_causal == 0
- * and N >= min_seq_len, else 0 (stay dense).  The default floor is passed
- * explicitly (SA_DEFAULT_MIN_SEQ_LEN); 0 means no floor, so every length
- * qualifies [SDN: 0 means no floor, the default is stated rather than hidden
- * behind a sentinel].  Negative values are reserved for a derived floor and
- * act as the default until one is defined.  Host only.
+ * default, the sparse/dense crossover measured there), and on the token
+ * mask or causal flag a block-only mask cannot combine with; a backend that
+ * takes the attention mask and the block mask together ("masked_block")
+ * serves masked calls].  has_token_mask is an sa_token_mask kind:
+ *   SA_TOKEN_MASK_NONE (0): no token mask;
+ *   SA_TOKEN_MASK_GENERAL (1): a mask that depends on the query token (any
+ *     [N][N] or per-query mask): declined, a block list cannot express it;
+ *   SA_TOKEN_MASK_KEY_PADDING (2): a key padding mask, [B][N]: served by
+ *     sa_block_sparse_attention_masked / sa_attention_run_masked, so it does
+ *     not decline.
+ * Returns 1 when is_self_attention != 0, the mask kind is NONE or
+ * KEY_PADDING, is_causal == 0 and N >= min_seq_len, else 0 (stay dense).
+ * The default floor is passed explicitly (SA_DEFAULT_MIN_SEQ_LEN); 0 means
+ * no floor, so every length qualifies [SDN: 0 means no floor, the default is
+ * stated rather than hidden behind a sentinel].  Negative values are
+ * reserved for a derived floor and act as the default until one is defined.
+ * Any other mask kind counts as GENERAL.  Host only.
  */
 #define SA_DEFAULT_MIN_SEQ_LEN 8192
+typedef enum { SA_TOKEN_MASK_NONE = 0, SA_TOKEN_MASK_GENERAL = 1, SA_TOKEN_MASK_KEY_PADDING = 2 } sa_token_mask;
 SA_API int sa_sparse_stage_gate(int N, int min_seq_len, int is_self_attention, int has_token_mask, int is_causal);
 
 /* Why the gate above declines [SDN stage paragraph: the stage records why it
@@ -319,6 +329,28 @@ SA_API sa_status sa_attention_run_gqa(const void* Q, const void* K, const void* 
 SA_API sa_status sa_dense_attention_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N,
                                         int d, float softmax_scale, void* O, void* ws, size_t ws_bytes,
                                         sa_stream_t stream);
+
+/*
+ * Token-level key mask inside the kept tiles [SDN "masked_block": a backend
+ * takes the attention mask and the block mask together].  key_mask is a
+ * device byte array [B][N], 16-byte aligned, nonzero where key n of batch b
+ * may be attended (a padding mask), or NULL for none.  Query row q of block
+ * i attends to key n only when n's block is in idx[b][h][i][0 .. counts) and
+ * key_mask[b][n] != 0; a row left with no key gets O = 0.  The mask is packed
+ * into one 64-bit word per (batch, key block) in the workspace (one small
+ * kernel), and the attention kernel applies it only to kept tiles whose word
+ * is neither all ones nor zero (a zero word skips the tile).  Other arguments
+ * as in the _gqa forms (H_kv = H for plain multi-head attention).
+ */
+SA_API sa_status sa_block_sparse_attention_masked(const void* Q, const void* K, const void* V, int B, int H,
+                                                  int H_kv, int N, int d, const int32_t* idx, const int32_t* counts,
+                                                  int cap, const uint8_t* key_mask, const uint8_t* head_mask,
+                                                  int min_active, float softmax_scale, void* O, void* ws,
+                                                  size_t ws_bytes, sa_stream_t stream);
+SA_API sa_status sa_attention_run_masked(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N,
+                                         int d, const uint8_t* key_mask, const uint8_t* head_mask, int min_active,
+                                         float softmax_scale, void* O, void* ws, size_t ws_bytes,
+                                         sa_stream_t stream);
 
 /*
  * sa_density [SDN "host sync": density is read back only when something

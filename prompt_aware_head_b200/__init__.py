@@ -79,6 +79,9 @@ _SIGS = {
     "sa_block_sparse_attention_gqa": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _I, _F, _P, _P, _SZ, _P], _I),
     "sa_attention_run_gqa": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _F, _P, _P, _SZ, _P], _I),
     "sa_dense_attention_gqa": ([_P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _SZ, _P], _I),
+    "sa_block_sparse_attention_masked": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _I, _F, _P, _P, _SZ, _P],
+                                         _I),
+    "sa_attention_run_masked": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _F, _P, _P, _SZ, _P], _I),
     "sa_density": ([_P, _I, _I, _I, _P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
                     ctypes.POINTER(sa_stats), _P, _SZ, _P], _I),
     "sa_workspace_size": ([_I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
@@ -185,6 +188,21 @@ def sa_budget_schedule(densities, n_cand: int) -> Tuple[np.ndarray, np.ndarray]:
 
 
 SA_DECLINE_NOT_SELF_ATTENTION, SA_DECLINE_TOKEN_MASK, SA_DECLINE_CAUSAL, SA_DECLINE_SHORT = 1, 2, 4, 8
+# Token mask kinds the gate tells apart: a general (query-dependent) mask declines; a key padding
+# mask [B, N] is served by the _masked attention calls.
+SA_TOKEN_MASK_NONE, SA_TOKEN_MASK_GENERAL, SA_TOKEN_MASK_KEY_PADDING = 0, 1, 2
+
+
+def _mask_kind(token_mask) -> int:
+    """None / False: no mask; "keys": a key padding mask; True or "general": any other token mask;
+    an int is passed through."""
+    if token_mask is None or token_mask is False:
+        return SA_TOKEN_MASK_NONE
+    if token_mask is True or token_mask == "general":
+        return SA_TOKEN_MASK_GENERAL
+    if token_mask == "keys":
+        return SA_TOKEN_MASK_KEY_PADDING
+    return int(token_mask)
 _DECLINE_NAMES = ((SA_DECLINE_NOT_SELF_ATTENTION, "not self attention"), (SA_DECLINE_TOKEN_MASK, "token mask"),
                   (SA_DECLINE_CAUSAL, "causal"), (SA_DECLINE_SHORT, "below the minimum length"))
 _declines_logged = set()
@@ -192,14 +210,15 @@ _log = logging.getLogger("prompt_aware_head_b200")
 
 
 def sa_sparse_stage_decline(N: int, min_seq_len: int = DEFAULT_MIN_SEQ_LEN, self_attention: bool = True,
-                            token_mask: bool = False, causal: bool = False) -> int:
-    """Bit set of the reasons the sparse stage declines a call (0: it does not)."""
+                            token_mask=None, causal: bool = False) -> int:
+    """Bit set of the reasons the sparse stage declines a call (0: it does not).
+    token_mask: None, "keys" (a key padding mask: served) or True / "general" (declined)."""
     return int(_lib.sa_sparse_stage_decline(int(N), int(min_seq_len), int(bool(self_attention)),
-                                            int(bool(token_mask)), int(bool(causal))))
+                                            _mask_kind(token_mask), int(bool(causal))))
 
 
 def sa_sparse_stage_gate(N: int, min_seq_len: int = DEFAULT_MIN_SEQ_LEN, self_attention: bool = True,
-                         token_mask: bool = False, causal: bool = False) -> bool:
+                         token_mask=None, causal: bool = False) -> bool:
     """True when a call should take the block-sparse path (host only).  A
     decline is logged once per (reasons, N), so a setting that cannot act is
     visible without repeating every call."""
@@ -323,6 +342,26 @@ def sa_dense_attention_gqa(Q, K, V, B: int, H: int, H_kv: int, N: int, d: int, s
     _check(_lib.sa_dense_attention_gqa(_addr(Q), _addr(K), _addr(V), B, H, H_kv, N, d,
                                        ctypes.c_float(softmax_scale), _addr(O), _addr(ws), ws_bytes,
                                        _stream(stream)), "sa_dense_attention_gqa")
+
+
+# Token-level key mask inside the kept tiles: key_mask is a device uint8 [B, N] (nonzero = may be attended).
+
+def sa_block_sparse_attention_masked(Q, K, V, B: int, H: int, H_kv: int, N: int, d: int, idx, counts, cap: int,
+                                     key_mask, head_mask, min_active: int, softmax_scale: float, O, ws, ws_bytes: int,
+                                     stream=None) -> None:
+    mptr, _keep = _host_mask(head_mask)
+    _check(_lib.sa_block_sparse_attention_masked(_addr(Q), _addr(K), _addr(V), B, H, H_kv, N, d, _addr(idx),
+                                                 _addr(counts), cap, _addr(key_mask), mptr, min_active,
+                                                 ctypes.c_float(softmax_scale), _addr(O), _addr(ws), ws_bytes,
+                                                 _stream(stream)), "sa_block_sparse_attention_masked")
+
+
+def sa_attention_run_masked(Q, K, V, B: int, H: int, H_kv: int, N: int, d: int, key_mask, head_mask,
+                            min_active: int, softmax_scale: float, O, ws, ws_bytes: int, stream=None) -> None:
+    mptr, _keep = _host_mask(head_mask)
+    _check(_lib.sa_attention_run_masked(_addr(Q), _addr(K), _addr(V), B, H, H_kv, N, d, _addr(key_mask), mptr,
+                                        min_active, ctypes.c_float(softmax_scale), _addr(O), _addr(ws), ws_bytes,
+                                        _stream(stream)), "sa_attention_run_masked")
 
 
 def sa_density(counts, B: int, H: int, nB: int, head_mask, ws, ws_bytes: int, stream=None):

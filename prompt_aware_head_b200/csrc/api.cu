@@ -37,6 +37,8 @@ WsLayout ws_layout(int B, int H, int N, int d) {
   off += align256(3 * BH * nB * sizeof(int32_t));
   w.totals = off;
   off += align256(BH * ((nB + 7) / 8) * 3 * sizeof(int32_t));
+  w.kmask = off;
+  off += align256(static_cast<size_t>(B) * nB * sizeof(uint64_t));
   w.total = off;
   return w;
 }
@@ -185,7 +187,7 @@ int sa_sparse_stage_decline(int N, int min_seq_len, int is_self_attention, int h
   const int min_len = min_seq_len >= 0 ? min_seq_len : SA_DEFAULT_MIN_SEQ_LEN;  // 0: no floor
   int why = 0;
   if (!is_self_attention) why |= SA_DECLINE_NOT_SELF_ATTENTION;
-  if (has_token_mask) why |= SA_DECLINE_TOKEN_MASK;
+  if (has_token_mask != SA_TOKEN_MASK_NONE && has_token_mask != SA_TOKEN_MASK_KEY_PADDING) why |= SA_DECLINE_TOKEN_MASK;
   if (is_causal) why |= SA_DECLINE_CAUSAL;
   if (N < min_len) why |= SA_DECLINE_SHORT;
   return why;
@@ -440,19 +442,27 @@ sa_status sa_attention_plan(const int32_t* idx, const int32_t* counts, int B, in
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
-sa_status sa_attention_run_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N, int d,
-                               const uint8_t* head_mask, int min_active, float softmax_scale, void* O, void* ws,
-                               size_t ws_bytes, sa_stream_t stream) {
+sa_status sa_attention_run_masked(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N, int d,
+                                  const uint8_t* key_mask, const uint8_t* head_mask, int min_active,
+                                  float softmax_scale, void* O, void* ws, size_t ws_bytes, sa_stream_t stream) {
   CallRange range("sa_attention_run");
   sa_status st = attention_args_ok(Q, K, V, O, B, H, H_kv, N, d, &softmax_scale);
   if (st != SA_OK) return st;
+  if (key_mask && !aligned16(key_mask)) return SA_ERR_INVALID_ARG;
   uint64_t bits = 0;
   if ((st = head_bits_of(head_mask, H, min_active, &bits)) != SA_OK) return st;
   if ((st = ws_ok(ws, ws_bytes, B, H, N, d)) != SA_OK) return st;
   DeviceInfo di;
   if ((st = check_device(&di)) != SA_OK) return st;
-  return from_cuda(launch_attention_run(Q, K, V, B, H, H_kv, N, d, bits, softmax_scale, O, ws,
+  return from_cuda(launch_attention_run(Q, K, V, B, H, H_kv, N, d, key_mask, bits, softmax_scale, O, ws,
                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sa_status sa_attention_run_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N, int d,
+                               const uint8_t* head_mask, int min_active, float softmax_scale, void* O, void* ws,
+                               size_t ws_bytes, sa_stream_t stream) {
+  return sa_attention_run_masked(Q, K, V, B, H, H_kv, N, d, nullptr, head_mask, min_active, softmax_scale, O, ws,
+                                 ws_bytes, stream);
 }
 
 sa_status sa_attention_run(const void* Q, const void* K, const void* V, int B, int H, int N, int d,
@@ -461,16 +471,26 @@ sa_status sa_attention_run(const void* Q, const void* K, const void* V, int B, i
   return sa_attention_run_gqa(Q, K, V, B, H, H, N, d, head_mask, min_active, softmax_scale, O, ws, ws_bytes, stream);
 }
 
+sa_status sa_block_sparse_attention_masked(const void* Q, const void* K, const void* V, int B, int H, int H_kv,
+                                           int N, int d, const int32_t* idx, const int32_t* counts, int cap,
+                                           const uint8_t* key_mask, const uint8_t* head_mask, int min_active,
+                                           float softmax_scale, void* O, void* ws, size_t ws_bytes,
+                                           sa_stream_t stream) {
+  sa_status st = attention_args_ok(Q, K, V, O, B, H, H_kv, N, d, &softmax_scale);
+  if (st != SA_OK) return st;
+  if (key_mask && !aligned16(key_mask)) return SA_ERR_INVALID_ARG;
+  if ((st = sa_attention_plan(idx, counts, B, H, N, d, cap, head_mask, min_active, ws, ws_bytes, stream)) != SA_OK)
+    return st;
+  return sa_attention_run_masked(Q, K, V, B, H, H_kv, N, d, key_mask, head_mask, min_active, softmax_scale, O, ws,
+                                 ws_bytes, stream);
+}
+
 sa_status sa_block_sparse_attention_gqa(const void* Q, const void* K, const void* V, int B, int H, int H_kv, int N,
                                         int d, const int32_t* idx, const int32_t* counts, int cap,
                                         const uint8_t* head_mask, int min_active, float softmax_scale, void* O,
                                         void* ws, size_t ws_bytes, sa_stream_t stream) {
-  sa_status st = attention_args_ok(Q, K, V, O, B, H, H_kv, N, d, &softmax_scale);
-  if (st != SA_OK) return st;
-  if ((st = sa_attention_plan(idx, counts, B, H, N, d, cap, head_mask, min_active, ws, ws_bytes, stream)) != SA_OK)
-    return st;
-  return sa_attention_run_gqa(Q, K, V, B, H, H_kv, N, d, head_mask, min_active, softmax_scale, O, ws, ws_bytes,
-                              stream);
+  return sa_block_sparse_attention_masked(Q, K, V, B, H, H_kv, N, d, idx, counts, cap, nullptr, head_mask,
+                                          min_active, softmax_scale, O, ws, ws_bytes, stream);
 }
 
 sa_status sa_block_sparse_attention(const void* Q, const void* K, const void* V, int B, int H, int N, int d,

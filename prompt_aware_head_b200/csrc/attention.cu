@@ -52,7 +52,16 @@ struct AttnArgs {
   __nv_bfloat16* O;
   float scale_log2;
   int* err;
+  // Token-level key mask inside kept tiles, or null: word [b][j] holds bit r
+  // set when key 64 j + r of batch b may be attended.
+  const unsigned long long* kmask;
 };
+
+// Mask word of the key block of union entry e for the item's batch (all
+// keys when there is no mask).
+__device__ __forceinline__ unsigned long long key_word(const AttnArgs& a, int bh, uint32_t e) {
+  return a.kmask ? __ldg(a.kmask + static_cast<size_t>(bh / a.H) * a.nB + (e & 0xFFFFu)) : ~0ull;
+}
 
 constexpr int kThreads = 384;  // Q/K producer, S issuer, 8 softmax warps, V producer, PV issuer
 constexpr float kRescaleThreshold = 8.0f;
@@ -590,16 +599,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY, l = 0.f;
       // this warp's union entry per step, prefetched one step ahead
       uint32_t en = cb < it.len ? load_entry(a, it, cb) : 0u;
+      unsigned long long wn = cb < it.len ? key_word(a, it.bh, en) : ~0ull;  // its key mask word, likewise
       for (int s = 0; s < nsteps; ++s, ++g) {
         const int sb = g & 1;
         const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
         const bool present = cb < nblk;        // this warp's key block exists in the step
         const uint32_t e = present ? en : 0u;
-        if (2 * s + 2 + cb < it.len) en = load_entry(a, it, 2 * s + 2 + cb);
+        const unsigned long long wm = wn;
+        if (2 * s + 2 + cb < it.len) {
+          en = load_entry(a, it, 2 * s + 2 + cb);
+          wn = key_word(a, it.bh, en);
+        }
         if (!warp_wait(&s_full[sb], (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
         tc_fence_after();
         if (sw == 0 && lane == 0) mbar_arrive(&k_empty[g % NK]);  // S_g done: its K stage is free
-        const bool bm = (e >> (16 + half)) & 1u;  // this half's query block selected the key block
+        // this half's query block selected the key block, and the key mask leaves some of its keys
+        const bool bm = ((e >> (16 + half)) & 1u) && wm != 0ull;
         uint32_t pk[32];
         float alpha = 1.f, sum = 0.f;
         bool rescale = false;
@@ -609,6 +624,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(s_col, x);
           tmem_ld32(s_col + 32, x + 32);
           tmem_wait_ld();
+          const bool partial = wm != ~0ull;  // the same for every row of the warp
+          if (partial) {  // masked keys take no part in the max and get probability 0
+#pragma unroll
+            for (int q = 0; q < 64; ++q)
+              if (!((wm >> q) & 1ull)) x[q] = 0xFF800000u;  // -inf
+          }
           float mv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int q = 0; q < 32; ++q)
@@ -627,6 +648,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           float sv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           float mv0 = 0.f, mv1 = 0.f;
           exp_half<false>(x, c, m, pk, sv, mv0, mv1);
+          if (partial) {  // exactly 0 for masked keys (the polynomial path floors 2^y at 2^-125)
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              pk[q] &= (((wm >> (2 * q)) & 1ull) ? 0x0000FFFFu : 0u) | (((wm >> (2 * q + 1)) & 1ull) ? 0xFFFF0000u : 0u);
+          }
           sum = sum8(sv);
         } else {
 #pragma unroll
@@ -717,6 +743,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tm, 512);
   }
+}
+
+// Packs a key mask of bytes, [B][N] (nonzero = may be attended), into one
+// 64-bit word per (batch, key block): bit r for key 64 j + r.  One thread per
+// word, four 16-byte loads each.
+__global__ void key_mask_words_kernel(const uint8_t* __restrict__ km, unsigned long long* __restrict__ words,
+                                      int n_words) {
+  grid_dep_wait();
+  const int w = blockIdx.x * blockDim.x + threadIdx.x;
+  if (w >= n_words) return;
+  const uint4* src = reinterpret_cast<const uint4*>(km + static_cast<size_t>(w) * 64);
+  unsigned long long bits = 0;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const uint4 u = __ldg(src + v);
+    const uint32_t parts[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        if ((parts[p] >> (8 * b)) & 0xFFu) bits |= 1ull << (16 * v + 4 * p + b);
+  }
+  words[w] = bits;
 }
 
 // Zero output for skipped heads.
@@ -818,11 +867,20 @@ static cudaError_t launch_attn(const void* Q, const void* K, const void* V, int 
 }
 
 cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int Hkv, int N, int d,
-                                 uint64_t head_bits, float scale, void* O, void* ws, cudaStream_t s) {
+                                 const uint8_t* key_mask, uint64_t head_bits, float scale, void* O, void* ws,
+                                 cudaStream_t s) {
   const int BH = B * H, nB = N / kBlock;
   const WsLayout wl = ws_layout(B, H, N, d);
   char* base = static_cast<char*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(base + wl.header);
+  unsigned long long* kmask = nullptr;
+  if (key_mask) {
+    kmask = reinterpret_cast<unsigned long long*>(base + wl.kmask);
+    const int n_words = B * nB;
+    cudaError_t e = launch_pdl(key_mask_words_kernel, dim3((n_words + 127) / 128), dim3(128), 0, s, key_mask,
+                               kmask, n_words);
+    if (e != cudaSuccess) return e;
+  }
   const uint64_t all = (H >= 64) ? ~0ull : ((1ull << H) - 1ull);
   if ((head_bits & all) != all) {
     const size_t per_head_vec = static_cast<size_t>(N) * d / 8;
@@ -844,6 +902,7 @@ cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, in
   args.O = static_cast<__nv_bfloat16*>(O);
   args.scale_log2 = scale * 1.4426950408889634f;
   args.err = &hdr->err;
+  args.kmask = kmask;
   return launch_attn(Q, K, V, BH, B * Hkv, N, d, args, s);
 }
 

@@ -49,6 +49,7 @@ struct WsLayout {
   size_t ulist = 0;         // int32 [3 strides][BH][nB][nB] union lists (j | bits << 16)
   size_t lens = 0;          // int32 [3 strides][BH][nB] union length per first block of a pair (-1: not a first)
   size_t totals = 0;        // int32 [BH][nB/8 rounded up][3] per-CTA partial sums of union lengths
+  size_t kmask = 0;         // uint64 [B][nB] key mask words (bit r: key 64 j + r may be attended)
   size_t total = 0;
 };
 WsLayout ws_layout(int B, int H, int N, int d);
@@ -78,6 +79,7 @@ cudaError_t launch_density(const int32_t* counts, int B, int H, int nB, uint64_t
 cudaError_t launch_attention_plan(const int32_t* idx, const int32_t* counts, int B, int H, int N, int d, int cap,
                                   uint64_t head_bits, void* ws, cudaStream_t s);
 cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int Hkv, int N, int d,
+                                 const uint8_t* key_mask,
                                  uint64_t head_bits, float scale, void* O, void* ws, cudaStream_t s);
 cudaError_t launch_dense_attention(const void* Q, const void* K, const void* V, int B, int H, int Hkv, int N,
                                    int d, float scale, void* O, void* ws, cudaStream_t s);

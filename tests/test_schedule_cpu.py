@@ -61,7 +61,11 @@ def test_stage_gate(sa):
     assert sa.sa_sparse_stage_gate(64, min_seq_len=0)             # 0: no floor, every length qualifies
     assert not sa.sa_sparse_stage_gate(8191, min_seq_len=-1)      # negative: reserved, the default floor for now
     assert not sa.sa_sparse_stage_gate(16896, self_attention=False)
-    assert not sa.sa_sparse_stage_gate(16896, token_mask=True)
+    assert not sa.sa_sparse_stage_gate(16896, token_mask=True)          # a general token mask declines
+    assert not sa.sa_sparse_stage_gate(16896, token_mask="general")
+    assert sa.sa_sparse_stage_gate(16896, token_mask="keys")              # a key padding mask is served
+    assert sa.sa_sparse_stage_decline(16896, token_mask=sa.SA_TOKEN_MASK_KEY_PADDING) == 0
+    assert sa.sa_sparse_stage_decline(16896, token_mask=7) == sa.SA_DECLINE_TOKEN_MASK  # unknown kinds: general
     assert not sa.sa_sparse_stage_gate(16896, causal=True)
 
 
