@@ -190,6 +190,31 @@ def test_realized_density_closed_form():
         assert da == pytest.approx(tiles / w.nB ** 2)
 
 
+def test_density_over_active_and_over_all_with_skipped_heads():
+    # joint layout, two batches of 24 heads with heads 5-8 skipped: every active head keeps 19969 tiles
+    # (P(P+C) + C(P+k)) and a skipped head none, so over the active heads the density is 19969 / nB^2 and over
+    # all heads 19969 * 20 / (24 nB^2) -- dividing either by the other head count fails one of the two
+    w = WORKLOADS["joint"]
+    H, B = 24, 2
+    cls = oracle.layout(list(w.segments), w.N)
+    hm = np.ones(H, np.uint8)
+    hm[5:9] = 0
+    sc = np.random.default_rng(5).standard_normal((B * H, w.nB, w.nB))
+    idx, counts = oracle.select(sc, cls, H, 0.3, hm)
+    assert int(counts.sum()) == 19969 * B * 20
+    da, dall = oracle.density(counts, H, w.nB, hm)
+    assert da == pytest.approx(19969 / w.nB ** 2, rel=1e-12)
+    assert dall == pytest.approx(19969 * 20 / (24 * w.nB ** 2), rel=1e-12)
+    # no mask: both are the same; every head skipped but one: over_all is 1/24 of over_active
+    da1, dall1 = oracle.density(counts, H, w.nB, None)
+    assert da1 == pytest.approx(dall1, rel=1e-12) and dall1 == pytest.approx(dall, rel=1e-12)
+    one = np.zeros(H, np.uint8)
+    one[3] = 1
+    _, c1 = oracle.select(sc, cls, H, 0.3, one)
+    a1, b1 = oracle.density(c1, H, w.nB, one)
+    assert a1 == pytest.approx(19969 / w.nB ** 2, rel=1e-12) and b1 == pytest.approx(a1 / 24, rel=1e-12)
+
+
 def test_min_active_heads_in_stack_masks():
     g = read_golden("crate_constants.txt")
     min_active = int(g["MIN_ACTIVE_HEADS"])
