@@ -220,23 +220,34 @@ SA_API sa_status sa_select_blocks(const sa_layout* L, const void* Q, const void*
  * this entry point exists for hosts that own all device memory and give
  * plugins no allocator, and for latency-critical code that must not call
  * cudaMalloc (which can synchronise the whole device).  It takes no
- * workspace: the pooled block means live in one fixed array of 16 MiB of
- * device memory inside the library, which every GPU that loads the library
- * holds until the process exits.  2 * B * H * nB * d * 4 bytes must fit in
- * it (e.g. B1 H24 N33280 d128 needs 12.8 MB); larger calls return
- * SA_ERR_WORKSPACE before anything is launched.  When scores_out is NULL the
- * scores are kept in the same array too, so the heads are then processed in
- * as many groups as that takes.  The call allocates nothing.
+ * workspace: its scratch (the pooled block means as tensor-core operand
+ * images, and the scores when scores_out is NULL) lives in one fixed array
+ * of 16 MiB of device memory inside the library, which every GPU that loads
+ * the library holds until the process exits.  The heads are processed in as
+ * many groups as that array needs.  The call is capped at 2 * B * H * nB * d
+ * * 4 <= 16 MiB (the fp32 block means of Q and K of every head at once; e.g.
+ * B1 H24 N33280 d128 needs 12.8 MB): a cap on the call's size, not its
+ * footprint, which grouping keeps within the array.  Larger calls return
+ * SA_ERR_WORKSPACE before anything is launched.  The call allocates nothing.
  * The first call on a device looks up the array's device address for that
  * device, so make that first call before any stream capture.  All calls
  * share the one array, which keeps the last call's contents (each call
  * overwrites what it reads); calls that overlap on the GPU (two streams, or
- * two host threads) race on it, so serialise them.  Arguments, outputs and
- * errors are otherwise those of sa_select_blocks.
+ * two host threads) race on it, so serialise them.  Arguments and outputs
+ * are otherwise those of sa_select_blocks; device-side errors are read with
+ * sa_check_noalloc (below) instead of sa_check.
  */
 SA_API sa_status sa_select_blocks_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int d,
                                           float density, const uint8_t* head_mask, int min_active,
                                           int32_t* idx, int32_t* counts, float* scores_out, sa_stream_t stream);
+
+/* The device-side errors of sa_select_blocks_noalloc, which has no workspace
+ * to record them in: its kernels set bits in an error word inside the same
+ * fixed array (one per device).  sa_check_noalloc synchronises `stream`,
+ * reads the current device's word, clears it, and returns SA_OK or the first
+ * error recorded since the last read (as sa_check does for a workspace).
+ * The word is shared by every call on the device, like the array. */
+SA_API sa_status sa_check_noalloc(sa_stream_t stream);
 
 /*
  * sa_pattern_mask [SDN "radial control"; GLO sliding window / dilated /
@@ -387,6 +398,12 @@ SA_API sa_status sa_debug_exp2(const float* y, float* out, int n, sa_stream_t st
  * so the next sa_check reports SA_ERR_TIMEOUT and the device stays usable.
  * Not on the hot path; for tests. */
 SA_API sa_status sa_debug_wait_timeout(void* ws, size_t ws_bytes, sa_stream_t stream);
+
+/* Diagnostic: records `status` (SA_ERR_BAD_INDEX or SA_ERR_TIMEOUT, else
+ * SA_ERR_INVALID_ARG) in the no-allocation path's error word of the current
+ * device with one small kernel, as a faulting selection kernel would, so the
+ * next sa_check_noalloc reports it.  Not on the hot path; for tests. */
+SA_API sa_status sa_debug_noalloc_error(int status, sa_stream_t stream);
 
 /* Library version string. */
 SA_API const char* sa_version(void);

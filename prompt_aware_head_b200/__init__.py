@@ -87,6 +87,8 @@ _SIGS = {
     "sa_workspace_size": ([_I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "sa_workspace_init": ([_P, _SZ, _P], _I),
     "sa_check": ([_P, _P], _I),
+    "sa_check_noalloc": ([_P], _I),
+    "sa_debug_noalloc_error": ([_I, _P], _I),
     "sa_debug_exp2": ([_P, _P, _I, _P], _I),
     "sa_debug_wait_timeout": ([_P, _SZ, _P], _I),
     "sa_status_string": ([_I], ctypes.c_char_p),
@@ -245,6 +247,12 @@ def sa_check(ws, stream=None) -> int:
     return int(_lib.sa_check(_addr(ws), _stream(stream)))
 
 
+def sa_check_noalloc(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device-side status
+    of sa_select_blocks_noalloc calls on the current device."""
+    return int(_lib.sa_check_noalloc(_stream(stream)))
+
+
 def sa_select_blocks(L: Layout, Q, K, B: int, H: int, d: int, density: float, head_mask, min_active: int,
                      idx, counts, scores_out, ws, ws_bytes: int, stream=None) -> None:
     mptr, _keep = _host_mask(head_mask)
@@ -377,6 +385,12 @@ def sa_debug_wait_timeout(ws, ws_bytes: int, stream=None) -> None:
     """Runs one kernel whose bounded wait runs out (about 2 s); the next
     sa_check reports SA_ERR_TIMEOUT."""
     _check(_lib.sa_debug_wait_timeout(_addr(ws), ws_bytes, _stream(stream)), "sa_debug_wait_timeout")
+
+
+def sa_debug_noalloc_error(status: int, stream=None) -> None:
+    """Records status in the no-allocation path's error word (test hook); the
+    next sa_check_noalloc reports it."""
+    _check(_lib.sa_debug_noalloc_error(int(status), _stream(stream)), "sa_debug_noalloc_error")
 
 
 def sa_debug_exp2(y, out, n: int, stream=None) -> None:

@@ -59,6 +59,10 @@ __global__ void wait_timeout_kernel(int* err) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, err);  // phase 0 never completes: runs out
 }
 
+// Diagnostic: records error bits in a device error word, as a kernel that
+// found a fault would.
+__global__ void set_error_kernel(int* err, int bits) { atomicOr(err, bits); }
+
 cudaError_t device_info(DeviceInfo* out) {
   static DeviceInfo cache[64];
   static std::mutex mu;
@@ -313,18 +317,31 @@ sa_status sa_workspace_init(void* ws, size_t ws_bytes, sa_stream_t stream) {
   return from_cuda(cudaMemsetAsync(ws, 0, sizeof(WsHeader), reinterpret_cast<cudaStream_t>(stream)));
 }
 
-sa_status sa_check(void* ws, sa_stream_t stream) {
-  if (!ws) return SA_ERR_WORKSPACE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+// Synchronises the stream, reads the device error word at `word`, clears it
+// when set, and maps its bits to a status (the first recorded kind).
+static sa_status read_and_clear_error(int* word, cudaStream_t s) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return SA_ERR_CUDA;
   int err = 0;
-  if (cudaMemcpy(&err, &static_cast<WsHeader*>(ws)->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return SA_ERR_CUDA;
-  if (err && cudaMemset(&static_cast<WsHeader*>(ws)->err, 0, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
+  if (cudaMemcpy(&err, word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SA_ERR_CUDA;
+  if (err && cudaMemset(word, 0, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
   if (err & kErrBadIndex) return SA_ERR_BAD_INDEX;
   if (err & kErrTimeout) return SA_ERR_TIMEOUT;
   if (err & kErrSmemAlign) return SA_ERR_UNSUPPORTED;
   return SA_OK;
+}
+
+sa_status sa_check(void* ws, sa_stream_t stream) {
+  if (!ws) return SA_ERR_WORKSPACE;
+  return read_and_clear_error(&static_cast<WsHeader*>(ws)->err, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_check_noalloc(sa_stream_t stream) {
+  DeviceInfo di;
+  sa_status st = check_device(&di);
+  if (st != SA_OK) return st;
+  int* word = nullptr;
+  if (noalloc_error_word(&word) != cudaSuccess) return SA_ERR_CUDA;
+  return read_and_clear_error(word, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // Key/value heads: at least one, and H a whole number of groups of them.
@@ -370,7 +387,8 @@ sa_status sa_select_blocks_noalloc_gqa(const sa_layout* L, const void* Q, const 
   uint64_t bits = 0;
   sa_status st = head_bits_of(head_mask, H, min_active, &bits);
   if (st != SA_OK) return st;
-  // the pooled block means (q-bar and k-bar, fp32) must fit the fixed scratch
+  // a cap on the call's size (not its footprint, which the head groups keep
+  // within the array): the fp32 block means of Q and K of every head at once
   const size_t need = 2ull * B * H * L->nB * d * sizeof(float);
   if (need > select_noalloc_limit()) return SA_ERR_WORKSPACE;
   DeviceInfo di;
@@ -552,6 +570,18 @@ sa_status sa_debug_wait_timeout(void* ws, size_t ws_bytes, sa_stream_t stream) {
   sa_status st = check_device(&di);
   if (st != SA_OK) return st;
   wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(&static_cast<WsHeader*>(ws)->err);
+  return from_cuda(cudaGetLastError());
+}
+
+sa_status sa_debug_noalloc_error(int bits, sa_stream_t stream) {
+  if (bits != SA_ERR_BAD_INDEX && bits != SA_ERR_TIMEOUT) return SA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  sa_status st = check_device(&di);
+  if (st != SA_OK) return st;
+  int* word = nullptr;
+  if (noalloc_error_word(&word) != cudaSuccess) return SA_ERR_CUDA;
+  set_error_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      word, bits == SA_ERR_BAD_INDEX ? kErrBadIndex : kErrTimeout);
   return from_cuda(cudaGetLastError());
 }
 

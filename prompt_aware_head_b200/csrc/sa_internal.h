@@ -66,6 +66,8 @@ cudaError_t launch_select(const sa_layout* L, const void* Q, const void* K, int 
                           cudaStream_t s);
 // Selection with its scratch in a fixed device array (no workspace).
 size_t select_noalloc_limit();
+// Device address of the no-allocation path's error word for the current device.
+cudaError_t noalloc_error_word(int** out);
 cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int Hkv, int d,
                                   int k, uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out,
                                   cudaStream_t s);

@@ -958,6 +958,16 @@ static cudaError_t noalloc_scratch(void** out) {
   return cudaSuccess;
 }
 
+// The error word the kernels of the no-allocation path record device-side
+// faults in: the last 256 bytes of the scratch array, zero at load.
+cudaError_t noalloc_error_word(int** out) {
+  void* scratch = nullptr;
+  const cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  *out = reinterpret_cast<int*>(static_cast<char*>(scratch) + kNoAllocScratchBytes - 256);
+  return cudaSuccess;
+}
+
 cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void* K, int B, int H, int Hkv, int d,
                                   int k, uint64_t head_bits, int32_t* idx, int32_t* counts, float* scores_out,
                                   cudaStream_t s) {
@@ -979,7 +989,9 @@ cudaError_t launch_select_noalloc(const sa_layout* L, const void* Q, const void*
   float* qimg = reinterpret_cast<float*>(base);
   float* kimg = reinterpret_cast<float*>(base + 2 * G * img);
   float* sc_scratch = reinterpret_cast<float*>(base + 4 * G * img);
-  int* err = reinterpret_cast<int*>(base + kNoAllocScratchBytes - 256);
+  int* err = nullptr;
+  e = noalloc_error_word(&err);
+  if (e != cudaSuccess) return e;
   for (int bh0 = 0; bh0 < BH; bh0 += G) {
     const int nbh = std::min(G, BH - bh0);
     float* sc = scores_out ? scores_out + static_cast<size_t>(bh0) * nB * nB : sc_scratch;

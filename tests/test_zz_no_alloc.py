@@ -3,8 +3,10 @@ device memory (hosts that own all device memory and give plugins no
 allocator, or latency-critical code that must not call cudaMalloc).  Its
 scratch is a fixed array inside the library; this test checks, through the C
 ABI, that two calls in a row give exactly what sa_select_blocks gives for the
-same inputs (lists bit-exact, scores identical), and that a call too large for
-the fixed array is refused before anything runs."""
+same inputs (lists bit-exact, scores identical), also with the scores kept in
+the array, that its device-side errors are reported by sa_check_noalloc and
+then cleared, and that a call beyond its size cap is refused before anything
+runs."""
 import numpy as np
 import pytest
 import torch
@@ -35,7 +37,7 @@ def _both(sa, w, seed, rho):
     counts = torch.full_like(ref.counts, -7)
     scores = torch.zeros_like(ref_scores)
     sa.sa_select_blocks_noalloc(L, q, k, w.B, w.H, w.d, rho, mask, w.min_active, idx, counts, scores)
-    torch.cuda.synchronize()
+    assert sa.sa_check_noalloc() == sa.SA_OK
     return ref, ref_scores, idx, counts, scores, mask
 
 
@@ -46,6 +48,38 @@ def test_noalloc_matches_workspace_selection_twice(sa):
         compare_lists(*ref.lists(), idx.cpu().numpy(), counts.cpu().numpy())
         for h in np.flatnonzero(mask):
             assert torch.equal(scores[:, h], ref_scores[:, h])
+
+
+def test_noalloc_lists_only_heads_in_groups(sa):
+    # no scores_out: the scores stay in the fixed array too, so the joint workload's 24 heads go through it in
+    # two groups (15 heads, then 9) -- the plain multi-head pooling path with scores in scratch
+    w = WORKLOADS["joint"]
+    Q, K, _ = make_qkv(w, seed=4)
+    q, k = dev_bf16(Q), dev_bf16(K)
+    L = sa.Layout(list(w.segments), w.N)
+    ref = Buffers(sa, w.B, w.H, w.N, w.d, L.cap)
+    sa.sa_select_blocks(L, q, k, w.B, w.H, w.d, 0.3, None, 0, ref.idx, ref.counts, None, ref.ws, ref.ws_bytes)
+    for _ in range(2):
+        idx = torch.full_like(ref.idx, -7)
+        counts = torch.full_like(ref.counts, -7)
+        sa.sa_select_blocks_noalloc(L, q, k, w.B, w.H, w.d, 0.3, None, 0, idx, counts, None)
+        assert sa.sa_check_noalloc() == sa.SA_OK
+        compare_lists(*ref.lists(), idx.cpu().numpy(), counts.cpu().numpy())
+
+
+def test_noalloc_device_errors_are_reported_then_cleared(sa):
+    # the path records device faults in an error word inside its fixed array; sa_check_noalloc reads and
+    # clears it (the word is set here by a one-thread kernel, as a faulting kernel would set it)
+    assert sa.sa_check_noalloc() == sa.SA_OK
+    sa.sa_debug_noalloc_error(sa.SA_ERR_TIMEOUT)
+    assert sa.sa_check_noalloc() == sa.SA_ERR_TIMEOUT
+    assert sa.sa_check_noalloc() == sa.SA_OK
+    sa.sa_debug_noalloc_error(sa.SA_ERR_BAD_INDEX)
+    assert sa.sa_check_noalloc() == sa.SA_ERR_BAD_INDEX
+    assert sa.sa_check_noalloc() == sa.SA_OK
+    with pytest.raises(sa.SAError) as e:
+        sa.sa_debug_noalloc_error(sa.SA_ERR_SHAPE)
+    assert e.value.status == sa.SA_ERR_INVALID_ARG
 
 
 def test_noalloc_refuses_sizes_beyond_its_scratch(sa):
