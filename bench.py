@@ -114,6 +114,18 @@ def job_value(flops_per_rank, ms_max, world):
 
 
 # ------------------------------------------------------------------ oracle (CPU) sample
+_INPUTS = {}
+
+
+def _inputs_once(w, seed):
+    """The workload's Q, K, V (all heads, layer 0), generated once per (workload, seed)."""
+    key = (w.name, w.N, w.H, w.d, seed)
+    if key not in _INPUTS:
+        _INPUTS.clear()
+        _INPUTS[key] = make_qkv(w, seed=seed)
+    return _INPUTS[key]
+
+
 def oracle_sample(w, rho, target_s=10.0, seed=0, g=1):
     """Times the fp64 oracle on whole heads of the workload (selection for the
     head, then attention for all its query rows) until about target_s of CPU
@@ -127,11 +139,10 @@ def oracle_sample(w, rho, target_s=10.0, seed=0, g=1):
     t_total = 0.0
     sel_s, att_s = 0.0, 0.0  # unscaled: every timed selection, every timed attention row
     done_heads, done_rows = 0, 0
+    Qa, Ka, Va = _inputs_once(w, seed)
     for h in heads:
-        Q, K, V = make_qkv(w, seed=seed, heads=[h])
-        if g > 1:
-            _, K, V = make_qkv(w, seed=seed, heads=[g * (h // g)])
-        Q, K, V = Q[:1], K[:1], V[:1]
+        hk = g * (h // g)  # the key/value head of h's group (itself without grouping)
+        Q, K, V = (np.ascontiguousarray(x[:1, hh:hh + 1]) for x, hh in ((Qa, h), (Ka, hk), (Va, hk)))
         t0 = time.perf_counter()
         sc = oracle.scores(oracle.pool(Q), oracle.pool(K)).reshape(-1, w.nB, w.nB)
         idx, cnt = oracle.select(sc, cls, 1, rho)
@@ -231,10 +242,13 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ traffic from the committed ncu summary
-def traffic_from_profile(kernel_src):
-    """dram bytes per launch recorded under profiles/ for the attention kernel, if
-    the kernel source has not changed since the capture (else None)."""
-    p = os.path.join(ROOT, "profiles", "sparse_attn_kernel_joint.md")
+def traffic_from_profile(kernel_src, workload="joint"):
+    """dram bytes per launch recorded under profiles/ for the attention kernel on
+    this workload, if the kernel source has not changed since the capture (else
+    None; also None when no workload is given)."""
+    if workload is None:
+        return None
+    p = os.path.join(ROOT, "profiles", "sparse_attn_kernel_%s.md" % workload)
     if not os.path.exists(p):
         return None
     digest = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
@@ -273,12 +287,19 @@ def run_ours(args):
     if H_kv < 1 or H % H_kv:
         raise SystemExit("--kv-heads must divide the workload's %d heads" % H)
     g = H // H_kv
-    mask = head_mask_for_layer(w)
-    Qh, Kh, Vh = make_qkv(w, seed=args.seed + rank)
-    if g > 1:
-        Kh, Vh = grouped_kv(Kh, Vh, g)
-    pin = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (Qh, Kh, Vh)]
-    Q, K, V = (p.to(dev, non_blocking=False) for p in pin)
+    # one step runs every layer of the workload (64 for the head-masked stack), each with its own inputs and
+    # head mask [HS AttentionMask: a mask per (layer, head)]
+    n_layers = min(args.layers or w.layers, w.layers)
+    masks = [head_mask_for_layer(w, l) for l in range(n_layers)]
+    pins, devs = [], []
+    for l in range(n_layers):
+        Qh, Kh, Vh = make_qkv(w, seed=args.seed + rank, layer=l)
+        if g > 1:
+            Kh, Vh = grouped_kv(Kh, Vh, g)
+        p = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (Qh, Kh, Vh)]
+        del Qh, Kh, Vh
+        pins.append(p)
+        devs.append(tuple(x.to(dev, non_blocking=False) for x in p))
     L = sa.Layout(list(w.segments), N)
     ws_bytes = sa.sa_workspace_size(B, H, N, d)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
@@ -288,7 +309,8 @@ def run_ours(args):
     O_host = torch.empty(O.shape, dtype=torch.bfloat16).pin_memory()
     stream = torch.cuda.current_stream(dev)
     sa.sa_workspace_init(ws, ws_bytes, stream)
-    in_bytes = (Q.numel() + K.numel() + V.numel()) * 2
+    layer_in_bytes = sum(x.numel() for x in devs[0]) * 2
+    in_bytes = n_layers * layer_in_bytes
     flush = in_bytes < 2 * L2_BYTES
     scratch = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev) if flush else None
     k_budget = sa.sa_budget(rho, L.n_cand)
@@ -300,9 +322,9 @@ def run_ours(args):
             if kind == SEG_PAD:
                 km[:, start:start + length] = 0
         km_dev = torch.from_numpy(km).to(dev)
-    n_masked = int(H - mask.sum())
 
-    def select(q, k):
+    def select(l, q, k):
+        mask = masks[l]
         if args.pattern == "content":
             sa.sa_select_blocks_gqa(L, q, k, B, H, H_kv, d, rho, mask, w.min_active, idx, counts, None, ws, ws_bytes,
                                     stream)
@@ -316,30 +338,39 @@ def run_ours(args):
                                window_tokens=512, n_global_blocks=8, stream=stream)
 
     def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        select(Q, K)
-        if ev is not None:
-            ev[1].record(stream)
-        sa.sa_attention_plan(idx, counts, B, H, N, d, L.cap, mask, w.min_active, ws, ws_bytes, stream)
-        if ev is not None:
-            ev[2].record(stream)
-        sa.sa_attention_run_masked(Q, K, V, B, H, H_kv, N, d, km_dev, mask, w.min_active, 0.0, O, ws, ws_bytes,
-                                   stream)
-        if ev is not None:
-            ev[3].record(stream)
+        """All layers; ev (if given) holds 4 events per layer: start, selected, planned, attended."""
+        for l in range(n_layers):
+            Q, K, V = devs[l]
+            e = ev[4 * l:4 * l + 4] if ev is not None else None
+            if e:
+                e[0].record(stream)
+            select(l, Q, K)
+            if e:
+                e[1].record(stream)
+            sa.sa_attention_plan(idx, counts, B, H, N, d, L.cap, masks[l], w.min_active, ws, ws_bytes, stream)
+            if e:
+                e[2].record(stream)
+            sa.sa_attention_run_masked(Q, K, V, B, H, H_kv, N, d, km_dev, masks[l], w.min_active, 0.0, O, ws,
+                                       ws_bytes, stream)
+            if e:
+                e[3].record(stream)
 
-    # selection (pool, scores, rank; one kernel for a pattern or a budget that
-    # covers every candidate), planner (rows, order), attention (+ zeroing of
-    # skipped heads)
-    launches_per_step = ((1 if dense_short or args.pattern != "content" else 3) + 2 + 1 + (1 if n_masked else 0)
-                         + (1 if km_dev is not None else 0))
+    # per layer: selection (pool, scores, rank; one kernel for a pattern or a budget that covers every
+    # candidate), planner (rows, order), attention (+ zeroing of skipped heads, + packing of a key mask)
+    launches_per_step = sum((1 if dense_short or args.pattern != "content" else 3) + 2 + 1
+                            + (1 if int(H - m.sum()) else 0) + (1 if km_dev is not None else 0) for m in masks)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     assert sa.sa_check(ws, stream) == sa.SA_OK
-    _, _, st = sa.sa_density(counts, B, H, w.nB, mask, ws, ws_bytes, stream)
-    tiles = st.tiles
+    # selected tiles of every layer (the lists of each layer, re-made once outside the timed region)
+    tiles = 0
+    tiles_per_layer = []
+    for l in range(n_layers):
+        select(l, *devs[l][:2])
+        _, _, st = sa.sa_density(counts, B, H, w.nB, masks[l], ws, ws_bytes, stream)
+        tiles += st.tiles
+        tiles_per_layer.append(st.tiles)
     flops_step = 4.0 * 64 * 64 * d * tiles
 
     uuid = None
@@ -348,7 +379,7 @@ def run_ours(args):
     except Exception:
         pass
     clocks = ClockSampler(uuid)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4 * n_layers)] for _ in range(args.steps)]
     clocks.start()
     if world > 1:
         dist.barrier()
@@ -361,39 +392,49 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    t_step = [e[0].elapsed_time(e[3]) for e in evs]
-    t_sel = [e[0].elapsed_time(e[1]) for e in evs]
-    t_plan = [e[1].elapsed_time(e[2]) for e in evs]
-    t_att = [e[2].elapsed_time(e[3]) for e in evs]
+    t_step = [e[0].elapsed_time(e[-1]) for e in evs]
+    t_sel = [sum(e[4 * l].elapsed_time(e[4 * l + 1]) for l in range(n_layers)) for e in evs]
+    t_plan = [sum(e[4 * l + 1].elapsed_time(e[4 * l + 2]) for l in range(n_layers)) for e in evs]
+    t_att = [sum(e[4 * l + 2].elapsed_time(e[4 * l + 3]) for l in range(n_layers)) for e in evs]
     ms_step = statistics.mean(t_step)
     ms_max = max_over_ranks(ms_step, dev)
     value = job_value(flops_step, ms_max, world)
     assert sa.sa_check(ws, stream) == sa.SA_OK
 
-    # dense baseline (same library, all heads, same inputs), and torch SDPA
+    # dense baseline (same library, all heads of every layer, same inputs), and torch SDPA
     dense_ms = sdpa_ms = None
     if not args.no_dense:
         Od = torch.empty_like(O)
+
+        def dense_all():
+            for l in range(n_layers):
+                Q, K, V = devs[l]
+                sa.sa_dense_attention_gqa(Q, K, V, B, H, H_kv, N, d, 0.0, Od, ws, ws_bytes, stream)
+
         for _ in range(3):
-            sa.sa_dense_attention_gqa(Q, K, V, B, H, H_kv, N, d, 0.0, Od, ws, ws_bytes, stream)
+            dense_all()
         de = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
         for a, b in de:
             if flush:
                 scratch.fill_(1.0)
             a.record(stream)
-            sa.sa_dense_attention_gqa(Q, K, V, B, H, H_kv, N, d, 0.0, Od, ws, ws_bytes, stream)
+            dense_all()
             b.record(stream)
         torch.cuda.synchronize()
         dense_ms = statistics.mean(a.elapsed_time(b) for a, b in de)
         try:
-            def f(q, k, v):
-                return torch.nn.functional.scaled_dot_product_attention(q, k, v, enable_gqa=g > 1)
+            def sdpa_all():
+                for l in range(n_layers):
+                    Q, K, V = devs[l]
+                    torch.nn.functional.scaled_dot_product_attention(Q, K, V, enable_gqa=g > 1)
             for _ in range(2):
-                f(Q, K, V)
+                sdpa_all()
             se = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(3)]
             for a, b in se:
+                if flush:
+                    scratch.fill_(1.0)
                 a.record(stream)
-                f(Q, K, V)
+                sdpa_all()
                 b.record(stream)
             torch.cuda.synchronize()
             sdpa_ms = statistics.mean(a.elapsed_time(b) for a, b in se)
@@ -401,57 +442,63 @@ def run_ours(args):
             sdpa_ms = None
         del Od
 
-    # End to end through the public API with host buffers (pinned): every step
-    # copies its Q, K, V in and its O out inside the timed region.  The copies
-    # are pipelined across steps as a serving loop would run them: step i's
-    # inputs go in on a copy stream while step i-1 computes, its O comes out on
-    # another copy stream while step i+1 computes (two device slots of Q/K/V
-    # and O; each slot is refilled only after the step that used it is done).
+    # End to end through the public API with host buffers (pinned): every layer of every step copies its Q, K,
+    # V in and its O out inside the timed region.  The copies are pipelined as a serving loop would run them:
+    # unit u's inputs go in on a copy stream while unit u-1 computes, its O comes out on another copy stream
+    # while unit u+1 computes (two device slots of Q/K/V and O; a slot is refilled only after the unit that
+    # used it is done).  A unit is one layer of one step.
     e2e_steps = max(1, min(args.steps, 10))
+    units = e2e_steps * n_layers
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    slots = [(Q, K, V, O), tuple(torch.empty_like(x) for x in (Q, K, V, O))]
-    in_done = [torch.cuda.Event() for _ in range(e2e_steps)]
-    comp_done = [torch.cuda.Event() for _ in range(e2e_steps)]
-    out_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    slots = [tuple(torch.empty_like(x) for x in devs[0]) + (O,),
+             tuple(torch.empty_like(x) for x in devs[0]) + (torch.empty_like(O),)]
+    in_done = [torch.cuda.Event() for _ in range(units)]
+    comp_done = [torch.cuda.Event() for _ in range(units)]
+    out_done = [torch.cuda.Event() for _ in range(units)]
     ee = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     torch.cuda.synchronize()
     ee[0].record(s_in)
-    for i in range(e2e_steps):
-        q, k, v, o = slots[i % 2]
-        if i >= 2:
-            s_in.wait_event(comp_done[i - 2])
+    for u in range(units):
+        l = u % n_layers
+        q, k, v, o = slots[u % 2]
+        if u >= 2:
+            s_in.wait_event(comp_done[u - 2])
         with torch.cuda.stream(s_in):
-            q.copy_(pin[0], non_blocking=True)
-            k.copy_(pin[1], non_blocking=True)
-            v.copy_(pin[2], non_blocking=True)
-        in_done[i].record(s_in)
-        stream.wait_event(in_done[i])
-        if i >= 2:
-            stream.wait_event(out_done[i - 2])
-        select(q, k)
-        sa.sa_block_sparse_attention_masked(q, k, v, B, H, H_kv, N, d, idx, counts, L.cap, km_dev, mask,
+            q.copy_(pins[l][0], non_blocking=True)
+            k.copy_(pins[l][1], non_blocking=True)
+            v.copy_(pins[l][2], non_blocking=True)
+        in_done[u].record(s_in)
+        stream.wait_event(in_done[u])
+        if u >= 2:
+            stream.wait_event(out_done[u - 2])
+        select(l, q, k)
+        sa.sa_block_sparse_attention_masked(q, k, v, B, H, H_kv, N, d, idx, counts, L.cap, km_dev, masks[l],
                                             w.min_active, 0.0, o, ws, ws_bytes, stream)
-        comp_done[i].record(stream)
-        s_out.wait_event(comp_done[i])
+        comp_done[u].record(stream)
+        s_out.wait_event(comp_done[u])
         with torch.cuda.stream(s_out):
             O_host.copy_(o, non_blocking=True)
-        out_done[i].record(s_out)
+        out_done[u].record(s_out)
     ee[1].record(s_out)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(ee[0].elapsed_time(ee[1]) / e2e_steps, dev)
+    assert sa.sa_check(ws, stream) == sa.SA_OK
     del slots
 
     pk, pk_kind = peaks()
     att_ms = statistics.mean(t_att)
     sel_ms = statistics.mean(t_sel)
     achieved = flops_step / (att_ms * 1e-3) / 1e12
-    traffic = traffic_from_profile(os.path.join(ROOT, "prompt_aware_head_b200", "csrc", "attention.cu"))
-    n_act = int(mask.sum())
-    n_kv_act = len({h // g for h in np.flatnonzero(mask)})  # key heads some active query head reads
+    traffic = traffic_from_profile(os.path.join(ROOT, "prompt_aware_head_b200", "csrc", "attention.cu"),
+                                   args.workload if n_layers == 1 and args.pattern == "content" else None)
+    n_act = sum(int(m.sum()) for m in masks)
+    # key heads some active query head reads, summed over layers
+    n_kv_act = sum(len({h // g for h in np.flatnonzero(m)}) for m in masks)
     # a control pattern reads no Q or K: only its lists count
     sel_bytes = ((1.0 * B * (n_act + n_kv_act) * N * d * 2 if args.pattern == "content" else 0.0)
                  + 4.0 * tiles + 4.0 * B * n_act * w.nB)
     sel_gbs = sel_bytes / (sel_ms * 1e-3) / 1e9
+    dense_flops = 4.0 * B * H * N * N * d * n_layers
     out = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -466,13 +513,15 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic (seeded; Q/K rank-8 sinusoidal position structure + noise, V ~ N(0,1); no weights)",
         "config": {
-            "workload": describe(w, rho, H_kv),
-            "B": B, "H": H, "H_kv": H_kv, "N": N, "d": d, "density_budget": rho, "lists": args.pattern,
-            "key_mask": "padding tokens masked inside kept tiles" if km_dev is not None else None,
+            "workload": describe(w, rho, H_kv) + (" x %d layers" % n_layers if n_layers > 1 else ""),
+            "B": B, "H": H, "H_kv": H_kv, "N": N, "d": d, "layers": n_layers, "density_budget": rho,
+            "lists": args.pattern,
+            "active_heads": n_act,
             "density_realized": round(tiles / (B * n_act * w.nB ** 2), 5),
             "selected_tiles": int(tiles),
             "l2": "flushed between steps (512 MB write outside the per-step events)" if flush
                   else "inputs larger than L2 (%.0f MB of Q/K/V)" % (in_bytes / 1e6),
+            "key_mask": "padding tokens masked inside kept tiles" if km_dev is not None else None,
             "parallelism": "replicas x%d (independent batches, no collective)" % world,
         },
         "breakdown_ms": {"select": round(sel_ms, 5), "plan": round(statistics.mean(t_plan), 5),
@@ -482,7 +531,9 @@ def run_ours(args):
         "speedup_vs_dense": round(dense_ms / ms_step, 3) if dense_ms else None,
         "attention_speedup_vs_dense": round(dense_ms / att_ms, 3) if dense_ms else None,
         "dense_ms": round(dense_ms, 5) if dense_ms else None,
-        "dense_tflops": round(4.0 * B * H * N * N * d / (dense_ms * 1e-3) / 1e12, 2) if dense_ms else None,
+        "dense_tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 2) if dense_ms else None,
+        "dense_roofline_frac": round(dense_flops / (dense_ms * 1e-3) / 1e12 / pk["bf16_tflops"], 4) if dense_ms
+        else None,
         "torch_sdpa_dense_ms": round(sdpa_ms, 5) if sdpa_ms else None,
         "speedup_vs_torch_sdpa": round(sdpa_ms / ms_step, 3) if sdpa_ms else None,
         "roofline": {
@@ -501,15 +552,22 @@ def run_ours(args):
             "frac": round(sel_gbs / pk["hbm_gbs"], 4), "algorithmic_bytes": int(sel_bytes),
         },
         "e2e": {"value": round(job_value(flops_step, e2e_ms, world), 3), "unit": UNIT,
-                "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(O.numel() * 2),
+                "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(O.numel() * 2 * n_layers),
                 "ms_per_step": round(e2e_ms, 4),
-                "copies": "pinned host buffers; step i+1's inputs in and step i-1's O out overlap step i"},
+                "copies": "pinned host buffers; unit u+1's inputs in and unit u-1's O out overlap unit u "
+                          "(a unit is one layer of one step)"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
+    if n_layers > 1:
+        out["per_layer_ms"] = {"step": round(ms_max / n_layers, 5), "select": round(sel_ms / n_layers, 5),
+                               "attention": round(att_ms / n_layers, 5),
+                               "dense": round(dense_ms / n_layers, 5) if dense_ms else None}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = oracle_sample(w, rho, target_s=args.cpu_seconds, seed=args.seed + rank, g=g)
         cb.pop("seconds", None)
+        if n_layers > 1:
+            cb["sample"] += "; layer 0 of %d" % n_layers
         out["cpu_baseline"] = cb
     if world > 1:
         dist.barrier()
@@ -637,6 +695,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0, help="input seed (rank r draws seed + r)")
     ap.add_argument("--pad-mask", action="store_true",
                     help="mask the layout's padding tokens as keys inside the kept tiles (token-level key mask)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers per step for a multi-layer workload (default: all of them, 64 for the stack)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
