@@ -592,7 +592,7 @@ def run_crossover(args):
     stream = torch.cuda.current_stream(dev)
     scratch = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     points = []
-    for N in (2048, 4096, 6144, 8192, 12288, 16384, 24576, 32768):
+    for N in (512, 1024, 1536, 2048, 3072, 4096, 6144, 8192, 12288, 16384, 24576, 32768):
         w = make_workload("joint", N=N, segments=(), grid=(N // 128, 128))
         B, H, d = w.B, w.H, w.d
         Q, K, V = (torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16) for x in make_qkv(w))

@@ -57,15 +57,18 @@ struct AttnArgs {
   const unsigned long long* kmask;
 };
 
-// Mask word of the key block of union entry e for the item's batch (all
-// keys when there is no mask).
+// Mask word of the key block of union entry e for the item's batch.  The
+// kernel is built twice: without a key mask every word is all ones at
+// compile time, so the unmasked kernel carries none of the masking code.
+template <bool kMask>
 __device__ __forceinline__ unsigned long long key_word(const AttnArgs& a, int bh, uint32_t e) {
-  return a.kmask ? __ldg(a.kmask + static_cast<size_t>(bh / a.H) * a.nB + (e & 0xFFFFu)) : ~0ull;
+  if constexpr (kMask) return __ldg(a.kmask + static_cast<size_t>(bh / a.H) * a.nB + (e & 0xFFFFu));
+  else return ~0ull;
 }
 
 constexpr int kThreads = 384;  // Q/K producer, S issuer, 8 softmax warps, V producer, PV issuer
-constexpr float kRescaleThreshold = 8.0f;
-constexpr uint32_t kBackoffNs = 40;            // producer / MMA poll back-off  // log2 units: rescale O when the max grows by > 2^8
+constexpr float kRescaleThreshold = 8.0f;       // log2 units: rescale O when the max grows by > 2^8
+constexpr uint32_t kBackoffNs = 40;            // producer poll back-off (ns)
 
 struct Item {
   int bh, i0, i1, len, off;
@@ -299,10 +302,13 @@ struct AttnSmem {
   static constexpr int kVBlock = 64 * D * 2;     // one V block, laid out [D/64 chunks][64 keys][128 B]
   static constexpr int kChunk = 128 * 128;       // one 64-column chunk of a 128-row tile
   // K and V live in separate rings: a K stage is free as soon as its S MMA
-  // completes, a V stage once its PV MMA does.  Three stages each cover the
-  // ~1 us latency of an L2-resident TMA load at d = 128 (224 KB in all).
-  static constexpr int kQBuf = (D == 128) ? 1 : 2;
-  static constexpr int kNK = (D == 128) ? 3 : 4;
+  // completes, a V stage once its PV MMA does.  Q is double-buffered, so the
+  // next item's Q tile lands during the current item (an item boundary no
+  // longer waits for it); at d = 128 that takes a K stage: Q 2 + K 2 + V 3
+  // tiles of 32 KB = 224 KB (V is read later in a step than K, so it keeps
+  // the deeper ring).
+  static constexpr int kQBuf = 2;
+  static constexpr int kNK = (D == 128) ? 2 : 4;
   static constexpr int kNV = (D == 128) ? 3 : 4;
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kQBuf * kTile;
@@ -317,7 +323,7 @@ struct AttnSmem {
   static_assert(kBytes <= kAlloc, "dynamic shared memory above the 227 KB per-CTA limit");
 };
 
-template <int D>
+template <int D, bool kMask>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
@@ -516,7 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
           const uint64_t bdesc = smem_desc_sw128(smem_u32(sm + S::kK + kst * S::kTile), 16, 1024);
           issue_qk<D>(tm + (g & 1) * 128, adesc, bdesc, idesc_bf16_f32(128, 64 * nblk, 0, 0));
-          tc_commit(&s_full[g & 1]);  // K stage kst is released by a softmax warp once S_g is complete
+          tc_commit(&s_full[g & 1]);
+          tc_commit(&k_empty[kst]);  // the S MMA has read the K stage
           if (s == nsteps - 1) tc_commit(&q_empty[qb]);
         }
         ++t;
@@ -599,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY, l = 0.f;
       // this warp's union entry per step, prefetched one step ahead
       uint32_t en = cb < it.len ? load_entry(a, it, cb) : 0u;
-      unsigned long long wn = cb < it.len ? key_word(a, it.bh, en) : ~0ull;  // its key mask word, likewise
+      unsigned long long wn = cb < it.len ? key_word<kMask>(a, it.bh, en) : ~0ull;  // its key mask word, likewise
       for (int s = 0; s < nsteps; ++s, ++g) {
         const int sb = g & 1;
         const int nblk = (2 * s + 1 < it.len) ? 2 : 1;
@@ -608,11 +615,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const unsigned long long wm = wn;
         if (2 * s + 2 + cb < it.len) {
           en = load_entry(a, it, 2 * s + 2 + cb);
-          wn = key_word(a, it.bh, en);
+          wn = key_word<kMask>(a, it.bh, en);
         }
         if (!warp_wait(&s_full[sb], (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
         tc_fence_after();
-        if (sw == 0 && lane == 0) mbar_arrive(&k_empty[g % NK]);  // S_g done: its K stage is free
         // this half's query block selected the key block, and the key mask leaves some of its keys
         const bool bm = ((e >> (16 + half)) & 1u) && wm != 0ull;
         uint32_t pk[32];
@@ -841,7 +847,7 @@ static bool make_map(CUtensorMap* map, const void* base, size_t rows, int d) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool kMask>
 static cudaError_t launch_attn_kernel(const void* Q, const void* K, const void* V, int BH, int BHkv, int N,
                                       const AttnArgs& args, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
@@ -853,17 +859,23 @@ static cudaError_t launch_attn_kernel(const void* Q, const void* K, const void* 
   if (e != cudaSuccess) return e;
   static int configured_dev_mask = 0;
   if (!(configured_dev_mask & (1 << (di.id & 31)))) {
-    e = cudaFuncSetAttribute(sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem<D>::kAlloc);
+    e = cudaFuncSetAttribute(sparse_attn_kernel<D, kMask>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnSmem<D>::kAlloc);
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << (di.id & 31);
   }
-  return launch_pdl(sparse_attn_kernel<D>, dim3(di.sm_count), dim3(kThreads), AttnSmem<D>::kAlloc, s, mq, mk, mv, args);
+  return launch_pdl(sparse_attn_kernel<D, kMask>, dim3(di.sm_count), dim3(kThreads), AttnSmem<D>::kAlloc, s, mq, mk,
+                    mv, args);
 }
 
 static cudaError_t launch_attn(const void* Q, const void* K, const void* V, int BH, int BHkv, int N, int d,
                                const AttnArgs& args, cudaStream_t s) {
-  if (d == 128) return launch_attn_kernel<128>(Q, K, V, BH, BHkv, N, args, s);
-  return launch_attn_kernel<64>(Q, K, V, BH, BHkv, N, args, s);
+  if (args.kmask) {
+    if (d == 128) return launch_attn_kernel<128, true>(Q, K, V, BH, BHkv, N, args, s);
+    return launch_attn_kernel<64, true>(Q, K, V, BH, BHkv, N, args, s);
+  }
+  if (d == 128) return launch_attn_kernel<128, false>(Q, K, V, BH, BHkv, N, args, s);
+  return launch_attn_kernel<64, false>(Q, K, V, BH, BHkv, N, args, s);
 }
 
 cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int Hkv, int N, int d,
