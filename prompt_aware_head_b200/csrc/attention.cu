@@ -1,6 +1,7 @@
 // Flash-style attention over selected (query block, key block) tiles on
 // sm_100a: tcgen05 MMA with TMEM accumulators, TMA-staged K/V tiles gathered
-// through the block lists, a persistent CTA per SM.
+// through the block lists, a persistent CTA per SM taking work items from an
+// atomic queue.
 //
 // What is computed follows the inferensys glossary ("block-sparse": only
 // connected (query block, key block) pairs are computed) and the SD.Next
@@ -55,6 +56,10 @@ struct AttnArgs {
   // Token-level key mask inside kept tiles, or null: word [b][j] holds bit r
   // set when key 64 j + r of batch b may be attended.
   const unsigned long long* kmask;
+  // Work queue: work[0] is the next item to hand out, work[1] counts the CTAs
+  // that have finished; the last CTA to finish resets both to 0.
+  int* work;
+  int queue;  // 1: items from the queue; 0: dealt by CTA index (small launches)
 };
 
 // Mask word of the key block of union entry e for the item's batch.  The
@@ -115,8 +120,32 @@ __device__ __forceinline__ uint32_t load_entry(const AttnArgs& a, const Item& it
   return static_cast<uint32_t>(a.ulist[it.off + pos]);
 }
 
+// Items are handed out through a queue (an atomic counter in the workspace):
+// CTA c starts on item c, then takes the next item when it is ready for one,
+// so CTAs that drew short items take more of them and all finish together.
+// The items stay in the planner's order (each head's longest item first, then
+// head-major, longest first within a head), so the CTAs still work through
+// one head's K / V at a time.  In each CTA the Q / K producer takes the
+// items and publishes each through a ring of kRing slots in shared memory;
+// the other roles read the ring in the same order.
+constexpr int kRing = 8;
+constexpr uint32_t kRingReaders = 11;  // V producer, two MMA issuers, eight softmax warps
+
+// The static deal of small launches (a few items per CTA, where the queue's
+// atomics and final fence cost more than the balance gains): pass r gives
+// CTA c item r G + c, or r G + G - 1 - c on odd passes.
 __device__ __forceinline__ int item_index(int r, int cta, int G) {
-  return r * G + ((r & 1) ? (G - 1 - cta) : cta);  // boustrophedon over the CTAs
+  return r * G + ((r & 1) ? (G - 1 - cta) : cta);
+}
+
+// Reader side of the ring: the r-th item of this CTA (total when none is left).
+__device__ __forceinline__ bool ring_take(int r, const int* ring, uint64_t* ring_full, uint64_t* ring_empty,
+                                          volatile int* abort_flag, int* err, int* k) {
+  const int slot = r & (kRing - 1);
+  if (!mbar_wait(&ring_full[slot], (r / kRing) & 1, abort_flag, err)) return false;
+  *k = ring[slot];
+  mbar_arrive(&ring_empty[slot]);
+  return true;
 }
 
 // ---------------------------------------------------------------- MMA issue
@@ -333,7 +362,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   if (pad + S::kBytes > static_cast<uint32_t>(S::kAlloc)) {  // uniform across the CTA: nothing started yet
-    if (threadIdx.x == 0) atomicOr(a.err, kErrSmemAlign);
+    if (threadIdx.x == 0) {
+      atomicOr(a.err, kErrSmemAlign);
+      if (a.queue && atomicAdd(a.work + 1, 1) == static_cast<int>(gridDim.x) - 1) {  // the last CTA resets the queue
+        atomicExch(a.work, 0);
+        atomicExch(a.work + 1, 0);
+      }
+    }
     return;
   }
   uint8_t* sm = smem_raw + pad;
@@ -348,11 +383,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_empty = k_full + NK;          // [NK] after the S MMA that read the stage
   uint64_t* v_full = k_empty + NK;          // [NV]
   uint64_t* v_empty = v_full + NV;          // [NV] after the PV MMA that read the stage
-  uint64_t* pair_x = v_empty + NV;          // [2 step parities][4 quads]: block-max exchange
-  uint64_t* pair_l = pair_x + 8;            // [4 quads]: row-sum exchange at the end of an item
+  uint64_t* pair_l = v_empty + NV;          // [4 quads]: row-sum exchange at the end of an item
   uint64_t* pair_g = pair_l + 4;            // [4 quads]: exchange slot released
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pair_g + 4);
+  uint64_t* ring_full = pair_g + 4;         // [kRing] the item in the slot is published
+  uint64_t* ring_empty = ring_full + kRing; // [kRing] every reader has taken it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ring_empty + kRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* ring = reinterpret_cast<int*>(tmem_slot + 2);  // [kRing] item indices
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -373,7 +410,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    for (int i = 0; i < 8; ++i) mbar_init(&pair_x[i], 2);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&ring_full[i], 1);
+      mbar_init(&ring_empty[i], kRingReaders);
+    }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&pair_l[i], 2);
       mbar_init(&pair_g[i], 2);
@@ -390,7 +430,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   grid_dep_wait();  // the work items come from the planner
   const uint32_t tm = *tmem_slot;
-  const int G = gridDim.x, cta = blockIdx.x;
   const int total = a.dense ? a.n_items_host : *reinterpret_cast<const volatile int*>(a.n_items_dev);
 
   if (warp == 0) {
@@ -400,8 +439,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       int k_phase[NK], q_phase[2] = {-1, -1};
       for (int i = 0; i < NK; ++i) k_phase[i] = -1;
       bool ok = true;
+      // The first item of CTA c is item c (no wait on the queue to start); the
+      // queue hands out the items after the first G.  Each take is made one
+      // item ahead of its use, so the atomic's latency hides behind the
+      // current item's loads (a taken index below total is always used).
+      const int G = static_cast<int>(gridDim.x);
+      int k_next = min(static_cast<int>(blockIdx.x), total);
       for (int r = 0; ok; ++r) {
-        const int k = item_index(r, cta, G);
+        int k;
+        if (a.queue) {  // publish the item to the other roles
+          const int slot = r & (kRing - 1);
+          if (r >= kRing && !mbar_wait(&ring_empty[slot], (r / kRing - 1) & 1, abort_flag, a.err, kBackoffNs)) {
+            ok = false;
+            break;
+          }
+          k = k_next;
+          ring[slot] = k;
+          mbar_arrive(&ring_full[slot]);
+          if (k < total) k_next = min(G + atomicAdd(a.work, 1), total);
+        } else {
+          k = min(item_index(r, static_cast<int>(blockIdx.x), G), total);
+        }
         if (k >= total) break;
         const Item it = load_item(a, k);
         const int nsteps = (it.len + 1) >> 1;
@@ -461,7 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < NV; ++i) v_phase[i] = -1;
       bool ok = true;
       for (int r = 0; ok; ++r) {
-        const int k = item_index(r, cta, G);
+        int k = min(item_index(r, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x)), total);
+        if (a.queue && !ring_take(r, ring, ring_full, ring_empty, abort_flag, a.err, &k)) { ok = false; break; }
         if (k >= total) break;
         const Item it = load_item(a, k);
         const int nsteps = (it.len + 1) >> 1;
@@ -506,7 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t g = 0, t = 0;
       bool ok = true;
       for (int r = 0; ok; ++r) {
-        const int k = item_index(r, cta, G);
+        int k = min(item_index(r, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x)), total);
+        if (a.queue && !ring_take(r, ring, ring_full, ring_empty, abort_flag, a.err, &k)) { ok = false; break; }
         if (k >= total) break;
         const Item it = load_item(a, k);
         const int nsteps = (it.len + 1) >> 1;
@@ -541,7 +601,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t g = 0;
       bool ok = true;
       for (int r = 0; ok; ++r) {
-        const int k = item_index(r, cta, G);
+        int k = min(item_index(r, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x)), total);
+        if (a.queue && !ring_take(r, ring, ring_full, ring_empty, abort_flag, a.err, &k)) { ok = false; break; }
         if (k >= total) break;
         const Item it = load_item(a, k);
         const int nsteps = (it.len + 1) >> 1;
@@ -587,7 +648,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t g = 0, t = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
-      const int k = item_index(r, cta, G);
+      int k = min(item_index(r, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x)), total);
+      if (a.queue) {  // every softmax warp reads the ring; each releases the slot once
+        const int slot = r & (kRing - 1);
+        if (!warp_wait(&ring_full[slot], (r / kRing) & 1, abort_flag, a.err)) { ok = false; break; }
+        k = ring[slot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ring_empty[slot]);
+      }
       if (k >= total) break;
       const Item it = load_item(a, k);
       const int nsteps = (it.len + 1) >> 1;
@@ -745,6 +813,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (a.queue && threadIdx.x == 0) {
+    __threadfence();  // this CTA's takes from the queue come before its count
+    if (atomicAdd(a.work + 1, 1) == static_cast<int>(gridDim.x) - 1) {  // the last CTA resets the queue
+      atomicExch(a.work, 0);
+      atomicExch(a.work + 1, 0);
+    }
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tm, 512);
@@ -878,6 +953,15 @@ static cudaError_t launch_attn(const void* Q, const void* K, const void* V, int 
   return launch_attn_kernel<64, false>(Q, K, V, BH, BHkv, N, args, s);
 }
 
+// The queue pays off from about 8 items per CTA (measured on the joint and
+// video workloads, 21 and 42 items per CTA: 4 % faster); below that (SDXL,
+// one layer of the stack: 3-5 items per CTA) the static deal is faster.
+int use_queue(long long items) {
+  DeviceInfo di;
+  if (device_info(&di) != cudaSuccess) return 1;
+  return items >= 8ll * di.sm_count ? 1 : 0;
+}
+
 cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, int B, int H, int Hkv, int N, int d,
                                  const uint8_t* key_mask, uint64_t head_bits, float scale, void* O, void* ws,
                                  cudaStream_t s) {
@@ -915,6 +999,8 @@ cudaError_t launch_attention_run(const void* Q, const void* K, const void* V, in
   args.scale_log2 = scale * 1.4426950408889634f;
   args.err = &hdr->err;
   args.kmask = kmask;
+  args.work = &hdr->next_item;
+  args.queue = use_queue(B * __builtin_popcountll(head_bits & all) * args.npairs_dense);
   return launch_attn(Q, K, V, BH, B * Hkv, N, d, args, s);
 }
 
@@ -936,6 +1022,8 @@ cudaError_t launch_dense_attention(const void* Q, const void* K, const void* V, 
   args.O = static_cast<__nv_bfloat16*>(O);
   args.scale_log2 = scale * 1.4426950408889634f;
   args.err = &hdr->err;
+  args.work = &hdr->next_item;
+  args.queue = use_queue(args.n_items_host);
   return launch_attn(Q, K, V, BH, B * Hkv, N, d, args, s);
 }
 

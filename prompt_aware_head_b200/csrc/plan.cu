@@ -126,17 +126,18 @@ __device__ __forceinline__ int best_stride_of(const int* partials, int nparts, i
 
 // Per head: the pairing stride with the smallest summed union; its pairs
 // ordered by union length, longest first (rank counting over unique keys),
-// written at the head's offset in the global item list (heads in order; the
-// offset is the closed-form pair count of the heads before).  Items point
-// into the chosen stride's union lists.
+// at closed-form offsets (the pair counts of the heads before) in the global
+// item list; with `front`, each active head's longest pair moves to the
+// front of the list (one per head, heads in order).  Items point into the
+// chosen stride's union lists.
 __global__ void __launch_bounds__(kOrderThreads) plan_order_kernel(const int* __restrict__ lens3,
                                                                    const int* __restrict__ partials, int nparts,
                                                                    int nB, int BH, int H, uint64_t head_bits,
-                                                                   int4* __restrict__ items,
+                                                                   int front, int4* __restrict__ items,
                                                                    int* __restrict__ n_items) {
   __shared__ uint32_t keys[kMaxBlocks];
   __shared__ int tot[kOrderHeads * 3];  // summed union lengths per (head, stride) when BH <= kOrderHeads
-  __shared__ int nkeys, base_sh, total_sh;
+  __shared__ int nkeys, base_sh, total_sh, act_sh, nact_sh;
   grid_dep_launch();  // the attention kernel may set up on the SMs this small grid leaves idle
   grid_dep_wait();
   const int bh = blockIdx.x, t = threadIdx.x;
@@ -145,6 +146,8 @@ __global__ void __launch_bounds__(kOrderThreads) plan_order_kernel(const int* __
     nkeys = 0;
     base_sh = 0;
     total_sh = 0;
+    act_sh = 0;
+    nact_sh = 0;
   }
   if (shared_sums) {  // all threads add up the per-CTA partial sums of every head
     for (int e = t; e < BH * 3; e += kOrderThreads) tot[e] = 0;
@@ -164,18 +167,31 @@ __global__ void __launch_bounds__(kOrderThreads) plan_order_kernel(const int* __
       if (tot[h * 3 + si] < tot[h * 3 + best]) best = si;
     return best;
   };
-  int my_base = 0, my_total = 0;
+  int my_base = 0, my_total = 0, my_act = 0, my_nact = 0;
   for (int h = t; h < BH; h += kOrderThreads) {
-    const int p = ((head_bits >> (h % H)) & 1ull) ? pairs_of(nB, stride_of(best_of(h))) : 0;
+    const bool on = (head_bits >> (h % H)) & 1ull;
+    const int p = on ? pairs_of(nB, stride_of(best_of(h))) : 0;
     my_total += p;
-    if (h < bh) my_base += p;
+    my_nact += on ? 1 : 0;
+    if (h < bh) {
+      my_base += p;
+      my_act += on ? 1 : 0;
+    }
   }
   if (my_base) atomicAdd(&base_sh, my_base);
   if (my_total) atomicAdd(&total_sh, my_total);
+  if (my_act) atomicAdd(&act_sh, my_act);
+  if (my_nact) atomicAdd(&nact_sh, my_nact);
   __syncthreads();
   if (bh == 0 && t == 0) *n_items = total_sh;
   if (!((head_bits >> (bh % H)) & 1ull)) return;
-  const int base = base_sh;
+  // With `front` (launches that take items from the work queue) every active
+  // head's longest item (rank 0: on the workloads with a pinned text block,
+  // the pair holding that block, dense over every non-dropped key block) goes
+  // to the front of the whole list, head by head, and the rest follow
+  // head-major, longest first within a head: the long items start first and
+  // the list ends on short ones.  Without it the list is plainly head-major.
+  const int base = base_sh, act = act_sh, nact = nact_sh;
   const int si = best_of(bh), s = stride_of(si);
   const size_t plane = static_cast<size_t>(BH) * nB;
   const int* lens = lens3 + si * plane + static_cast<size_t>(bh) * nB;
@@ -196,7 +212,7 @@ __global__ void __launch_bounds__(kOrderThreads) plan_order_kernel(const int* __
     v.y = a | ((b < 0 ? kNoBlock : b) << 16);
     v.z = 0xFFFF - static_cast<int>(k >> 16);
     v.w = static_cast<int>((si * plane + static_cast<size_t>(bh) * nB + a) * nB);
-    items[base + rank] = v;
+    items[front ? (rank == 0 ? act : nact + (base - act) + (rank - 1)) : base + rank] = v;
   }
 }
 
@@ -213,8 +229,9 @@ cudaError_t launch_attention_plan(const int32_t* idx, const int32_t* counts, int
   cudaError_t e = launch_pdl(plan_rows_kernel, dim3(nparts, BH), dim3(256), 0, s, idx, counts, nB, cap, H, head_bits,
                              ulist, lens, partials, &hdr->err);
   if (e != cudaSuccess) return e;
+  const int front = use_queue(static_cast<long long>(B) * __builtin_popcountll(head_bits) * ((nB + 1) / 2));
   return launch_pdl(plan_order_kernel, dim3(BH), dim3(kOrderThreads), 0, s, static_cast<const int*>(lens),
-                    static_cast<const int*>(partials), nparts, nB, BH, H, head_bits, items, &hdr->n_items);
+                    static_cast<const int*>(partials), nparts, nB, BH, H, head_bits, front, items, &hdr->n_items);
 }
 
 }  // namespace sa

@@ -32,7 +32,9 @@ struct WsHeader {
   int err;                   // sticky error bits
   int n_items;               // attention work items written by the planner
   unsigned long long tiles;  // density accumulator
-  int pad[60];
+  int next_item;             // attention work queue: next item to hand out
+  int ctas_done;             // attention work queue: CTAs finished (the last resets both)
+  int pad[58];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 

@@ -77,6 +77,10 @@ cudaError_t launch_pattern(const sa_layout* L, int kind, int W, int G, int r, in
 cudaError_t launch_density(const int32_t* counts, int B, int H, int nB, uint64_t head_bits, void* ws,
                            unsigned long long* host_tiles, cudaStream_t s);
 
+// Whether the attention kernel takes its items from the work queue (1) or
+// deals them by CTA index (0), from the number of items of the launch.
+int use_queue(long long items);
+
 // Work plan (plan.cu) and attention launchers (attention.cu).
 cudaError_t launch_attention_plan(const int32_t* idx, const int32_t* counts, int B, int H, int N, int d, int cap,
                                   uint64_t head_bits, void* ws, cudaStream_t s);
