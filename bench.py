@@ -8,8 +8,13 @@ tiles.  Metric: effective TFLOP/s = 4 * 64 * 64 * d * (selected tiles) / step
 time, i.e. 4*B*H_active*N^2*d*density / t.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload joint|sdxl|video|stack|tiny]
-                  [--pattern content|radial|window] [--kv-heads H_kv]
+                  [--pattern content|radial|random|window] [--kv-heads H_kv] [--no-graph]
   python bench.py --impl reference ...     # the fp64 CPU oracle on a bounded sample
+
+Timing: each step (every layer) is captured once as a CUDA graph and
+replayed, K replays timed with CUDA events (--no-graph: eager launches);
+the stage times (selection, plan, attention kernel) come from a second run
+of K steps launched eagerly with events between the stages.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own
 independent batch (seed = rank); value = all ranks' flops / max-over-ranks
@@ -323,37 +328,52 @@ def run_ours(args):
                 km[:, start:start + length] = 0
         km_dev = torch.from_numpy(km).to(dev)
 
-    def select(l, q, k):
+    def select(l, q, k, st=None):
         mask = masks[l]
+        st = st or stream
         if args.pattern == "content":
             sa.sa_select_blocks_gqa(L, q, k, B, H, H_kv, d, rho, mask, w.min_active, idx, counts, None, ws, ws_bytes,
-                                    stream)
+                                    st)
         elif args.pattern == "radial":
-            sa.sa_pattern_mask(L, sa.SA_PAT_RADIAL, B, H, rho, mask, w.min_active, idx, counts, stream=stream)
+            sa.sa_pattern_mask(L, sa.SA_PAT_RADIAL, B, H, rho, mask, w.min_active, idx, counts, stream=st)
         elif args.pattern == "random":
-            sa.sa_pattern_mask(L, sa.SA_PAT_RANDOM, B, H, rho, mask, w.min_active, idx, counts, stream=stream,
+            sa.sa_pattern_mask(L, sa.SA_PAT_RANDOM, B, H, rho, mask, w.min_active, idx, counts, stream=st,
                                seed=rank)
         else:
             sa.sa_pattern_mask(L, sa.SA_PAT_WINDOW_GLOBAL, B, H, rho, mask, w.min_active, idx, counts,
-                               window_tokens=512, n_global_blocks=8, stream=stream)
+                               window_tokens=512, n_global_blocks=8, stream=st)
 
-    def step(ev=None):
-        """All layers; ev (if given) holds 4 events per layer: start, selected, planned, attended."""
+    def step(ev=None, st=None):
+        """All layers on stream st; ev (if given) holds 4 events per layer: start, selected, planned, attended."""
+        st = st or stream
         for l in range(n_layers):
             Q, K, V = devs[l]
             e = ev[4 * l:4 * l + 4] if ev is not None else None
             if e:
-                e[0].record(stream)
-            select(l, Q, K)
+                e[0].record(st)
+            select(l, Q, K, st)
             if e:
-                e[1].record(stream)
-            sa.sa_attention_plan(idx, counts, B, H, N, d, L.cap, masks[l], w.min_active, ws, ws_bytes, stream)
+                e[1].record(st)
+            sa.sa_attention_plan(idx, counts, B, H, N, d, L.cap, masks[l], w.min_active, ws, ws_bytes, st)
             if e:
-                e[2].record(stream)
+                e[2].record(st)
             sa.sa_attention_run_masked(Q, K, V, B, H, H_kv, N, d, km_dev, masks[l], w.min_active, 0.0, O, ws,
-                                       ws_bytes, stream)
+                                       ws_bytes, st)
             if e:
-                e[3].record(stream)
+                e[3].record(st)
+
+    def captured(fn):
+        """fn() captured once into a CUDA graph on a side stream (the library's calls take that stream)."""
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=cap):
+            fn(cap)
+        stream.wait_stream(cap)
+        for _ in range(2):
+            gr.replay()
+        torch.cuda.synchronize()
+        return gr
 
     # per layer: selection (pool, scores, rank; one kernel for a pattern or a budget that covers every
     # candidate), planner (rows, order), attention (+ zeroing of skipped heads, + packing of a key mask)
@@ -367,7 +387,7 @@ def run_ours(args):
     tiles = 0
     tiles_per_layer = []
     for l in range(n_layers):
-        select(l, *devs[l][:2])
+        select(l, *devs[l][:2], stream)
         _, _, st = sa.sa_density(counts, B, H, w.nB, masks[l], ws, ws_bytes, stream)
         tiles += st.tiles
         tiles_per_layer.append(st.tiles)
@@ -378,24 +398,54 @@ def run_ours(args):
         uuid = str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         pass
+    # The step (every layer) is captured once into a CUDA graph and replayed: a serving loop repeats the same
+    # launches every step, and the graph takes the host's launch path out of the timed region.  The step time
+    # comes from replays of that graph (events around each replay: an event record inside a graph breaks the
+    # programmatic-dependent-launch overlap of the kernels it separates).  The stage times (the attention
+    # kernel's among them, for the roofline) come from a second run of as many steps launched eagerly with
+    # events at the stage boundaries.
+    graph = captured(lambda st: step(None, st)) if not args.no_graph else None
     clocks = ClockSampler(uuid)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4 * n_layers)] for _ in range(args.steps)]
+    outer = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
+    def stage_times(e):
+        return (e[0].elapsed_time(e[-1]),
+                sum(e[4 * l].elapsed_time(e[4 * l + 1]) for l in range(n_layers)),
+                sum(e[4 * l + 1].elapsed_time(e[4 * l + 2]) for l in range(n_layers)),
+                sum(e[4 * l + 2].elapsed_time(e[4 * l + 3]) for l in range(n_layers)))
+
+    def eager_steps():
+        for i in range(args.steps):
+            if flush:
+                scratch.fill_(float(i))  # 512 MB write between steps, outside the per-step events
+            step(evs[i])
+
     clocks.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    for i in range(args.steps):
-        if flush:
-            scratch.fill_(float(i))  # 512 MB write between steps, outside the per-step events
-        step(evs[i])
+    if graph is not None:
+        for i in range(args.steps):
+            if flush:
+                scratch.fill_(float(i))
+            outer[i][0].record(stream)
+            graph.replay()
+            outer[i][1].record(stream)
+    else:
+        eager_steps()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    if graph is not None:  # the stage-time run
+        eager_steps()
+        torch.cuda.synchronize()
+        t_step = [a.elapsed_time(b) for a, b in outer]
     clk = clocks.stop()
-    t_step = [e[0].elapsed_time(e[-1]) for e in evs]
-    t_sel = [sum(e[4 * l].elapsed_time(e[4 * l + 1]) for l in range(n_layers)) for e in evs]
-    t_plan = [sum(e[4 * l + 1].elapsed_time(e[4 * l + 2]) for l in range(n_layers)) for e in evs]
-    t_att = [sum(e[4 * l + 2].elapsed_time(e[4 * l + 3]) for l in range(n_layers)) for e in evs]
+    stage_rows = [stage_times(e) for e in evs]
+    if graph is None:
+        t_step = [r[0] for r in stage_rows]
+    _, t_sel, t_plan, t_att = (list(x) for x in zip(*stage_rows))
     ms_step = statistics.mean(t_step)
     ms_max = max_over_ranks(ms_step, dev)
     value = job_value(flops_step, ms_max, world)
@@ -406,35 +456,41 @@ def run_ours(args):
     if not args.no_dense:
         Od = torch.empty_like(O)
 
-        def dense_all():
+        def dense_all(st=None):
             for l in range(n_layers):
                 Q, K, V = devs[l]
-                sa.sa_dense_attention_gqa(Q, K, V, B, H, H_kv, N, d, 0.0, Od, ws, ws_bytes, stream)
+                sa.sa_dense_attention_gqa(Q, K, V, B, H, H_kv, N, d, 0.0, Od, ws, ws_bytes, st or stream)
 
         for _ in range(3):
             dense_all()
+        if graph is not None:  # launched the same way as the sparse step
+            dgraph = captured(dense_all)
+            dense_run = dgraph.replay
+        else:
+            dense_run = dense_all
         de = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
         for a, b in de:
             if flush:
                 scratch.fill_(1.0)
             a.record(stream)
-            dense_all()
+            dense_run()
             b.record(stream)
         torch.cuda.synchronize()
         dense_ms = statistics.mean(a.elapsed_time(b) for a, b in de)
         try:
-            def sdpa_all():
+            def sdpa_all(st=None):
                 for l in range(n_layers):
                     Q, K, V = devs[l]
                     torch.nn.functional.scaled_dot_product_attention(Q, K, V, enable_gqa=g > 1)
             for _ in range(2):
                 sdpa_all()
+            sdpa_run = captured(sdpa_all).replay if graph is not None else sdpa_all
             se = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(3)]
             for a, b in se:
                 if flush:
                     scratch.fill_(1.0)
                 a.record(stream)
-                sdpa_all()
+                sdpa_run()
                 b.record(stream)
             torch.cuda.synchronize()
             sdpa_ms = statistics.mean(a.elapsed_time(b) for a, b in se)
@@ -523,6 +579,9 @@ def run_ours(args):
                   else "inputs larger than L2 (%.0f MB of Q/K/V)" % (in_bytes / 1e6),
             "key_mask": "padding tokens masked inside kept tiles" if km_dev is not None else None,
             "parallelism": "replicas x%d (independent batches, no collective)" % world,
+            "launch": "each step captured once as a CUDA graph and replayed (dense and SDPA likewise); stage "
+                      "times from a second run of as many steps launched eagerly with events between the stages"
+                      if graph is not None else "eager launches",
         },
         "breakdown_ms": {"select": round(sel_ms, 5), "plan": round(statistics.mean(t_plan), 5),
                          "attention": round(att_ms, 5)},
@@ -604,17 +663,31 @@ def run_crossover(args):
         counts = torch.zeros((B, H, w.nB), dtype=torch.int32, device=dev)
         O = torch.empty_like(Q)
 
-        def sparse():
-            sa.sa_select_blocks(L, Q, K, B, H, d, rho, None, 0, idx, counts, None, ws, ws_bytes, stream)
+        def sparse(st=None):
+            sa.sa_select_blocks(L, Q, K, B, H, d, rho, None, 0, idx, counts, None, ws, ws_bytes, st or stream)
             sa.sa_block_sparse_attention(Q, K, V, B, H, N, d, idx, counts, L.cap, None, 0, 0.0, O, ws, ws_bytes,
-                                         stream)
+                                         st or stream)
 
-        def dense():
-            sa.sa_dense_attention(Q, K, V, B, H, N, d, 0.0, O, ws, ws_bytes, stream)
+        def dense(st=None):
+            sa.sa_dense_attention(Q, K, V, B, H, N, d, 0.0, O, ws, ws_bytes, st or stream)
+
+        def as_graph(fn):  # both sides launched the same way as the bench's steps
+            cap = torch.cuda.Stream(dev)
+            cap.wait_stream(stream)
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cap):
+                fn(cap)
+            stream.wait_stream(cap)
+            return gr
 
         ms = []
+        graphs = []
         for fn in (sparse, dense):
             for _ in range(args.warmup):
+                fn()
+            if not args.no_graph:
+                graphs.append(as_graph(fn))
+                fn = graphs[-1].replay
                 fn()
             ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)]
@@ -627,6 +700,8 @@ def run_crossover(args):
             ms.append(statistics.mean(a.elapsed_time(b) for a, b in ev))
         assert sa.sa_check(ws, stream) == sa.SA_OK
         points.append((N, ms[0], ms[1]))
+        del graphs
+        torch.cuda.synchronize()
         L.release()
         del Q, K, V, O, ws, idx, counts
     n_star, kind = crossover(points)
@@ -636,7 +711,8 @@ def run_crossover(args):
         "warmup": args.warmup, "dtype": "bf16", "data": "synthetic (seeded)",
         "config": {"workload": "B1 H24 d128, image tokens only (rows of 128), density %.2f" % rho,
                    "l2": "flushed before every timed call (512 MB write outside the events)",
-                   "sparse": "sa_select_blocks + sa_block_sparse_attention", "dense": "sa_dense_attention"},
+                   "sparse": "sa_select_blocks + sa_block_sparse_attention", "dense": "sa_dense_attention",
+                   "launch": "each side captured as a CUDA graph and replayed" if not args.no_graph else "eager"},
         "points": [{"N": n, "sparse_ms": round(a, 5), "dense_ms": round(b, 5), "speedup": round(b / a, 3)}
                    for n, a, b in points],
     }), flush=True)
@@ -699,6 +775,8 @@ def main():
                     help="layers per step for a multi-layer workload (default: all of them, 64 for the stack)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch each step's kernels eagerly instead of replaying a captured CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--crossover", action="store_true",
                     help="instead of the step benchmark: the sequence length from which the sparse step beats dense "
