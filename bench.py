@@ -363,11 +363,13 @@ def run_ours(args):
                 e[3].record(st)
 
     def captured(fn):
-        """fn() captured once into a CUDA graph on a side stream (the library's calls take that stream)."""
+        """fn() captured once into a CUDA graph on a side stream (the library's calls take that stream).
+        Thread-local capture: other threads of the process (the NCCL watchdog under torchrun) keep
+        calling CUDA while this one captures."""
         cap = torch.cuda.Stream(dev)
         cap.wait_stream(stream)
         gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=cap):
+        with torch.cuda.graph(gr, stream=cap, capture_error_mode="thread_local"):
             fn(cap)
         stream.wait_stream(cap)
         for _ in range(2):
@@ -675,7 +677,7 @@ def run_crossover(args):
             cap = torch.cuda.Stream(dev)
             cap.wait_stream(stream)
             gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr, stream=cap):
+            with torch.cuda.graph(gr, stream=cap, capture_error_mode="thread_local"):
                 fn(cap)
             stream.wait_stream(cap)
             return gr
