@@ -712,12 +712,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           // Running max: set by the first selected block, raised again only
           // when it grows by more than 2^8 (then O_cb is rescaled); otherwise
           // the stale max is kept (exact after the final division by the sum).
-          if (m == -INFINITY) {
-            m = mx;
-          } else if (mx > m + kRescaleThreshold) {
-            alpha = ex2(m - mx);
-            m = mx;
-            rescale = true;
+          {  // as selects (no per-row branch): the exponential is taken in every row
+            const bool first = m == -INFINITY;
+            const bool grow = !first && mx > m + kRescaleThreshold;
+            const float a_ = ex2(m - mx);
+            alpha = grow ? a_ : 1.f;
+            rescale = grow;
+            m = (first || grow) ? mx : m;
           }
           float sv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           float mv0 = 0.f, mv1 = 0.f;
