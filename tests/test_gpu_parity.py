@@ -218,6 +218,22 @@ def test_attention_parity_joint_every_row(sa):
     print("joint rho=0.3 every row: max-abs %.3g mean-abs %.3g" % (mx, mean))
 
 
+def test_attention_parity_d64_work_queue(sa):
+    # d = 64 with enough items for the work queue (4 x 10 heads x 32 pairs = 1280 items, at least 8 per CTA
+    # on 148 SMs; SDXL itself has 640 and takes the static deal): 5 % of the rows, seeded, plus the first and
+    # last row of every head
+    w = make_workload("sdxl", B=4)
+    Q, K, V = make_qkv(w, seed=21)
+    L, buf, _ = _select(sa, w, Q, K, 0.3, None, 0, want_scores=False)
+    O = _attention(sa, w, Q, K, V, buf, None, 0)
+    idx, cnt = buf.lists()
+    edges = [bh * w.N + n for bh in range(w.B * w.H) for n in (0, w.N - 1)]
+    rows = sample_rows(w.B, w.H, w.N, 0.05, seed=4, must=edges)
+    ref = oracle.attention(Q, K, V, w.H, idx, cnt, rows=rows)
+    mx, mean = check_attention(host_f64(O).reshape(-1, w.d)[rows], ref, _live_rows(cnt, None, w.H, w.N)[rows])
+    print("sdxl x4 batches (work queue): max-abs %.3g mean-abs %.3g" % (mx, mean))
+
+
 def _pin_rows(w):
     """Flat row ids of every query row in a pinned block, over every head."""
     cls = oracle.layout(list(w.segments), w.N)
