@@ -62,6 +62,28 @@ def describe(w, rho, H_kv=None):
         (", head mask %d of %d" % (int(head_mask_for_layer(w).sum()), w.H)) if w.head_mask or w.mask_runs else "")
 
 
+def paired_tiles(idx, counts, head_mask, H, nB):
+    """64 x 64 tiles the attention kernel computes for these lists: the planner pairs query blocks (a, a + s)
+    with a // s even, s = 1, 2 or 4 per head (the smallest summed union, the smaller s on ties), and each pair
+    walks the union of its two lists with a 128-row tile (two 64 x 64 tiles per union entry).  Host-side
+    restatement of the planner's pairing, for reporting."""
+    idx = np.asarray(idx).reshape(-1, nB, idx.shape[-1])
+    cnt = np.asarray(counts).reshape(-1, nB)
+    BH = cnt.shape[0]
+    M = np.zeros((BH, nB, nB), bool)
+    b_ix, i_ix, e_ix = np.nonzero(np.arange(idx.shape[-1])[None, None, :] < cnt[..., None])
+    M[b_ix, i_ix, idx[b_ix, i_ix, e_ix]] = True
+    active = np.ones(BH, bool) if head_mask is None else np.tile(np.asarray(head_mask, bool), BH // H)
+    best = None
+    for s in (1, 2, 4):
+        a = np.array([i for i in range(nB) if (i // s) % 2 == 0])
+        b = a + s
+        partner = np.where((b < nB)[None, :, None], M[:, np.minimum(b, nB - 1)], False)
+        u = (M[:, a] | partner).sum(axis=(1, 2))
+        best = u if best is None else np.minimum(best, u)
+    return int(2 * best[active].sum())
+
+
 def grouped_kv(K, V, g):
     """K and V of the first head of each group of g query heads: the shared
     key/value heads of a grouped-query layout ([B, H / g, N, d])."""
@@ -388,11 +410,13 @@ def run_ours(args):
     # selected tiles of every layer (the lists of each layer, re-made once outside the timed region)
     tiles = 0
     tiles_per_layer = []
+    computed = 0
     for l in range(n_layers):
         select(l, *devs[l][:2], stream)
         _, _, st = sa.sa_density(counts, B, H, w.nB, masks[l], ws, ws_bytes, stream)
         tiles += st.tiles
         tiles_per_layer.append(st.tiles)
+        computed += paired_tiles(idx.cpu().numpy(), counts.cpu().numpy(), masks[l], H, w.nB)
     flops_step = 4.0 * 64 * 64 * d * tiles
 
     uuid = None
@@ -577,6 +601,9 @@ def run_ours(args):
             "active_heads": n_act,
             "density_realized": round(tiles / (B * n_act * w.nB ** 2), 5),
             "selected_tiles": int(tiles),
+            "computed_tiles": computed,  # 64 x 64 tiles the paired 128-row walk computes (effective TFLOP/s counts
+                                         # only the selected ones): pairing efficiency = selected / computed
+            "pairing_efficiency": round(tiles / computed, 4) if computed else None,
             "l2": "flushed between steps (512 MB write outside the per-step events)" if flush
                   else "inputs larger than L2 (%.0f MB of Q/K/V)" % (in_bytes / 1e6),
             "key_mask": "padding tokens masked inside kept tiles" if km_dev is not None else None,

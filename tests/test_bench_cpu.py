@@ -101,3 +101,33 @@ def test_crossover_interpolates_in_log_n():
     assert bench.crossover([(2048, 1.0, 1.2), (4096, 1.0, 3.0)]) == (2048.0, "at or below")
     assert bench.crossover([(2048, 2.0, 1.0), (4096, 2.0, 1.5)]) == (None, "above")
     assert bench.crossover([(8192, 1.0, 1.0)]) == (8192.0, "at or below")  # equal times count as a win
+
+
+def test_paired_tiles_matches_brute_force():
+    """bench.paired_tiles restates the planner's pairing (strides 1, 2, 4; smallest summed union, the smaller
+    stride on ties; two 64 x 64 tiles per union entry): checked against sets on random lists."""
+    import numpy as np
+    import bench
+    rng = np.random.default_rng(0)
+    for trial in range(20):
+        B, H = 2, 3
+        nB = int(rng.integers(1, 40))
+        cnt = rng.integers(0, nB + 1, size=(B, H, nB)).astype(np.int32)
+        idx = np.full((B, H, nB, nB), -1, np.int32)
+        for b in range(B):
+            for h in range(H):
+                for i in range(nB):
+                    idx[b, h, i, :cnt[b, h, i]] = np.sort(rng.choice(nB, cnt[b, h, i], replace=False))
+        mask = rng.integers(0, 2, H).astype(bool) if trial % 2 else None
+        want = 0
+        for b in range(B):
+            for h in range(H):
+                if mask is not None and not mask[h]:
+                    continue
+                sets = [set(idx[b, h, i, :cnt[b, h, i]].tolist()) for i in range(nB)]
+                per_stride = []
+                for s in (1, 2, 4):
+                    per_stride.append(sum(len(sets[a] | (sets[a + s] if a + s < nB else set()))
+                                          for a in range(nB) if (a // s) % 2 == 0))
+                want += 2 * min(per_stride)
+        assert bench.paired_tiles(idx, cnt, mask, H, nB) == want
