@@ -251,6 +251,8 @@ sa_status sa_build_layout(const sa_segment* segs, int nseg, int N, int block, sa
     if (L->cls[b] == kPin) ++L->n_pin;
     if (L->cls[b] == kDrop) ++L->n_drop;
     if (L->cls[b] == kSparse) rank[b] = r++;
+    if (L->cls[b] == kPin) L->pin_bits[b >> 5] |= 1u << (b & 31);
+    if (L->cls[b] == kSparse) L->sparse_bits[b >> 5] |= 1u << (b & 31);
   }
   L->n_cand = r;
   L->cap = L->nB - L->n_drop;

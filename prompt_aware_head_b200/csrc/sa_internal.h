@@ -16,6 +16,10 @@ struct sa_layout {
   int device = -1;
   uint8_t* d_cls = nullptr;         // device [nB] block classes
   int32_t* d_sparse_rank = nullptr; // device [nB]: index among SPARSE blocks, -1 otherwise
+  // block classes as bit masks over 32-block words (bit b of word c: block
+  // 32 c + b); blocks past nB are in neither (DROP)
+  uint32_t pin_bits[32] = {};
+  uint32_t sparse_bits[32] = {};
   int refcount = 0;
 };
 

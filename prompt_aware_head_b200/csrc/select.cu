@@ -609,69 +609,78 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(const __grid_constant_
 }
 
 // ============================================================== ranking rows
+// The layout's block classes as bit masks, passed by value (constant
+// memory): no per-CTA load of the classes before the scores can be read.
+struct ClassBits {
+  uint32_t pin[32], sparse[32];
+};
+
 // One warp per query block row (head bh = bh0 + slot) of the scores
 // score_tc_kernel wrote ([slot][nB][nB]): the pins,
 // the diagonal (it outranks every score) and the top k - 1 other sparse
 // candidates by the bucket select; the list goes out in ascending order.
-// Rows of skipped heads get empty lists.
+// Rows of skipped heads get empty lists.  Both of a warp's rows have their
+// scores loaded at the start, so the second row's load latency hides behind
+// the first row's selection.
 template <int NC>
 __global__ void __launch_bounds__(128, NC <= 17 ? 8 : 4) rank_rows_kernel(const float* __restrict__ scores,
-                                                           const uint8_t* __restrict__ cls_g, int nB, int H,
+                                                           const __grid_constant__ ClassBits cb, int nB, int H,
                                                            uint64_t head_bits, int k, int cap,
                                                            int32_t* __restrict__ idx, int32_t* __restrict__ counts,
                                                            int bh0) {
   __shared__ uint32_t hist[4][256];
   __shared__ uint32_t memk[4][32];
-  __shared__ uint8_t cls[32 * NC];
-  __shared__ uint32_t pin_m[NC], sparse_m[NC], drop_m[NC];  // class masks of key blocks 32c + lane
   grid_dep_wait();
-  for (int j = threadIdx.x; j < nB; j += 128) cls[j] = cls_g[j];
-  __syncthreads();
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, slot = blockIdx.y, bh = bh0 + slot;
-  for (int c = w; c < NC; c += 4) {
-    const int j = 32 * c + lane;
-    const uint8_t cj = j < nB ? cls[j] : static_cast<uint8_t>(kDrop);
-    const uint32_t pm = __ballot_sync(0xffffffffu, cj == kPin), sm = __ballot_sync(0xffffffffu, cj == kSparse);
-    if (lane == 0) {
-      pin_m[c] = pm;
-      sparse_m[c] = sm;
-      drop_m[c] = ~(pm | sm);
-    }
-  }
-  __syncthreads();
   const bool active_head = (head_bits >> (bh % H)) & 1ull;
+  // row rr's sparse candidates' scores (0 elsewhere); both rows up front where
+  // the registers allow (NC <= 9, up to 288 blocks), else each row in turn
+  constexpr bool kBoth = NC <= 9;
+  float sc[2][NC];
+  auto load_row = [&](int rr) {
+    const int i = blockIdx.x * 8 + rr * 4 + w;
+    const bool sparse_row = active_head && i < nB && ((cb.sparse[i >> 5] >> (i & 31)) & 1u);
+    const float* srow = scores + (static_cast<size_t>(slot) * nB + i) * nB + lane;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const bool sp = (cb.sparse[c] >> lane) & 1u;
+      sc[rr][c] = (sparse_row && sp && 32 * c + lane != i) ? __ldg(srow + 32 * c) : 0.f;
+    }
+  };
+  load_row(0);
+  if (kBoth) load_row(1);
+#pragma unroll
   for (int rr = 0; rr < 2; ++rr) {  // two rows per warp: one wave covers every row
     const int i = blockIdx.x * 8 + rr * 4 + w;
     if (i >= nB) return;
+    if (!kBoth && rr == 1) load_row(1);
     const size_t row = static_cast<size_t>(bh) * nB + i;
     if (!active_head) {
       if (lane == 0) counts[row] = 0;
       continue;
     }
-    const uint8_t ci = cls[i];
+    const bool row_pin = (cb.pin[i >> 5] >> (i & 31)) & 1u;
+    const bool row_sparse = (cb.sparse[i >> 5] >> (i & 31)) & 1u;
     uint32_t keep = 0;
-    if (ci == kPin) {
+    if (row_pin) {
 #pragma unroll
-      for (int c = 0; c < NC; ++c) keep |= ((~drop_m[c] >> lane) & 1u) << c;
-    } else if (ci == kSparse) {
-      float sc[NC];
+      for (int c = 0; c < NC; ++c) keep |= (((cb.pin[c] | cb.sparse[c]) >> lane) & 1u) << c;
+    } else if (row_sparse) {
       uint32_t cand = 0, diag = 0;
-      const float* srow = scores + (static_cast<size_t>(slot) * nB + i) * nB + lane;
 #pragma unroll
       for (int c = 0; c < NC; ++c) {
-        keep |= ((pin_m[c] >> lane) & 1u) << c;
-        const bool sp = (sparse_m[c] >> lane) & 1u;
+        keep |= ((cb.pin[c] >> lane) & 1u) << c;
+        const bool sp = (cb.sparse[c] >> lane) & 1u;
         const bool dg = 32 * c + lane == i;
         diag |= (sp && dg ? 1u : 0u) << c;
         cand |= (sp && !dg ? 1u : 0u) << c;
-        sc[c] = (sp && !dg) ? __ldg(srow + 32 * c) : 0.f;
       }
       if (k >= 1) {
         keep |= diag;
         const int kk = k - 1;
         const int ncand = __reduce_add_sync(0xffffffffu, __popc(cand));
         if (kk >= ncand) keep |= cand;
-        else if (kk > 0) keep |= warp_topk_bucket<NC>(sc, cand, kk, hist[w], memk[w]);
+        else if (kk > 0) keep |= warp_topk_bucket<NC>(sc[rr], cand, kk, hist[w], memk[w]);
       }
     }
     const int n = warp_emit<NC>(keep, idx + row * cap);
@@ -816,8 +825,11 @@ static cudaError_t ensure_smem(F* kernel, size_t bytes, bool* configured, std::m
 template <int NC>
 static cudaError_t launch_rank_t(const float* scores, const sa_layout* L, int bh0, int nbh, int H, uint64_t head_bits,
                                  int k, int32_t* idx, int32_t* counts, cudaStream_t s) {
-  return launch_pdl(rank_rows_kernel<NC>, dim3((L->nB + 7) / 8, nbh), dim3(128), 0, s, scores,
-                    static_cast<const uint8_t*>(L->d_cls), L->nB, H, head_bits, k, L->cap, idx, counts, bh0);
+  ClassBits cb;
+  std::memcpy(cb.pin, L->pin_bits, sizeof cb.pin);
+  std::memcpy(cb.sparse, L->sparse_bits, sizeof cb.sparse);
+  return launch_pdl(rank_rows_kernel<NC>, dim3((L->nB + 7) / 8, nbh), dim3(128), 0, s, scores, cb, L->nB, H,
+                    head_bits, k, L->cap, idx, counts, bh0);
 }
 
 static cudaError_t launch_rank(int nc, const float* scores, const sa_layout* L, int bh0, int nbh, int H,
